@@ -1,0 +1,230 @@
+"""fp64 CPU oracle for the exact attention forward pass (test infrastructure).
+
+Test infrastructure only: imported by the tests, ``__graft_entry__.smoke()``
+and the CPU-baseline / reference arm of ``bench.py``; never by the product path.
+It shares no code, header, table or constant with the CUDA library.
+
+What it computes (the plain definition, materialising S and P):
+
+* Page "Flash attention optimization" (aicomputerinstitute.com), section
+  "Attention is not slow because of arithmetic": for Q, K, V in R^{N x d},
+  S = Q K^T / sqrt(d), P = softmax(S) row-wise, O = P V.  The 1/sqrt(d) factor
+  is the caller's ``scale`` (default 1/sqrt(d)).
+* Same page, section "Worked example: online softmax by hand": the direct
+  softmax subtracts the row's global maximum before exponentiating, then
+  normalises by the sum of exponentials.
+* Causal mask (the ``is_causal=True`` flag of the page "FlashAttention: The GPU
+  Memory Hack That Changed Everything", section "Integration: It's
+  Everywhere"): key j is allowed for query i iff j <= i.  Masked scores are
+  -inf, so their weight exp(-inf - M) is exactly 0.
+* The saved per-row statistic (section "Sizing a tile, and why the backward
+  pass recomputes instead of storing" keeps the row max m and sum l):
+  exported as LSE_i = M_i + ln(sum_j exp(S_ij - M_i)), natural-log units,
+  scale included.
+
+The two online-softmax row functions restate, in fp64, the recurrence of the
+"The fix: tile the computation, never materialize the full matrix" section
+(block-local max, then scale_old / scale_new) and the running-max form of the
+first page's "The Tiling Strategy" pseudocode.  They exist only so the
+self-tests can check that tiling reaches the direct result; the oracle proper
+is the direct (materialising) definition.
+
+Parity is pinned by the CPU tests (worked example, exercise 1, closed forms,
+invariants, brute force and an independent library routine); nothing here is
+"parity unpinned".
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# Input conversion
+# ---------------------------------------------------------------------------
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """Exact conversion of raw bfloat16 bit patterns (uint16) to float64.
+
+    A bfloat16 is the upper 16 bits of an IEEE binary32; shifting the pattern
+    left by 16 gives that binary32 exactly, and binary32 -> binary64 is exact.
+    """
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def _as_f64(x) -> np.ndarray:
+    """Accept a numpy array or a CPU torch tensor (any real dtype) -> float64."""
+    if hasattr(x, "detach"):  # torch tensor: go through float32, exact for bf16/fp16/fp32
+        import torch
+
+        x = x.detach().to("cpu")
+        if x.dtype != torch.float64:
+            x = x.to(torch.float32)
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Direct (materialising) definition
+# ---------------------------------------------------------------------------
+
+def softmax_rows_fp64(S: np.ndarray):
+    """Row softmax of a score block with global-max subtraction.
+
+    Returns (P, M, Z): P = exp(S - M) / Z row-wise, M the row max and
+    Z = sum exp(S - M).  A row's masked entries are -inf and get weight 0.
+    """
+    M = np.max(S, axis=1, keepdims=True)
+    E = np.exp(S - M)
+    Z = np.sum(E, axis=1, keepdims=True)
+    return E / Z, M[:, 0], Z[:, 0]
+
+
+def attention_rows_fp64(q_bh, k_bh, v_bh, rows, causal: bool, scale: float):
+    """O and LSE for selected query rows of one (batch, head).
+
+    q_bh, k_bh, v_bh: (N, d) float64.  rows: 1-D int array of query indices.
+    Materialises the full score rows S[rows, :] and P[rows, :] (all N keys),
+    then O = P V.  Returns (O (len(rows), d), LSE (len(rows),)).
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    N = k_bh.shape[0]
+    S = scale * (q_bh[rows] @ k_bh.T)                       # S = Q K^T * scale
+    if causal:
+        keys = np.arange(N, dtype=np.int64)
+        S = np.where(keys[None, :] <= rows[:, None], S, -np.inf)   # allowed iff j <= i
+    P, M, Z = softmax_rows_fp64(S)                          # P = softmax(S)
+    O = P @ v_bh                                            # O = P V
+    LSE = M + np.log(Z)
+    return O, LSE
+
+
+def attention_fp64(q, k, v, causal: bool = False, scale: float | None = None,
+                   row_chunk: int = 512):
+    """Exact attention forward in float64 for (B, H, N, d) inputs.
+
+    Materialises S and P one chunk of ``row_chunk`` query rows at a time (rows
+    are independent, so chunking changes no result; it bounds host memory for
+    N = 32768).  Returns (O (B,H,N,d) float64, LSE (B,H,N) float64).
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    if q.ndim != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one (B, H, N, d) shape")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.empty((B, H, N, d), dtype=np.float64)
+    LSE = np.empty((B, H, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, N, row_chunk):
+                r1 = min(N, r0 + row_chunk)
+                rows = np.arange(r0, r1)
+                O[b, h, r0:r1], LSE[b, h, r0:r1] = attention_rows_fp64(
+                    q[b, h], k[b, h], v[b, h], rows, causal, scale)
+    return O, LSE
+
+
+# ---------------------------------------------------------------------------
+# Tiled forms (self-test companions, never the oracle)
+# ---------------------------------------------------------------------------
+
+def online_softmax_row_blockmax(scores, values, block: int):
+    """One query row, tiled, with each block's exponentials taken relative to
+    that block's own max and merged with scale_old = exp(m_old - m_new) and
+    scale_new = exp(m_block - m_new) (page "Flash attention optimization",
+    section "The fix: tile the computation, never materialize the full
+    matrix").  ``values`` is (n,) or (n, d).  Returns (O, m, l, trace) where
+    trace lists the running (m, l, acc) after each block.
+    """
+    s = np.asarray(scores, dtype=np.float64)
+    vals = np.asarray(values, dtype=np.float64)
+    n = s.shape[0]
+    m = -np.inf
+    l = 0.0
+    acc = np.zeros(vals.shape[1:], dtype=np.float64)
+    trace = []
+    for start in range(0, n, block):
+        sb = s[start:start + block]
+        vb = vals[start:start + block]
+        m_block = np.max(sb)
+        p = np.exp(sb - m_block)
+        l_block = np.sum(p)
+        acc_block = np.tensordot(p, vb, axes=(0, 0))
+        m_new = max(m, m_block)
+        # With m = -inf on the first block this factor is exp(-inf) = 0:
+        # the empty running state is discarded without a special case.
+        scale_old = np.exp(m - m_new)
+        scale_new = np.exp(m_block - m_new)
+        l = l * scale_old + l_block * scale_new
+        acc = acc * scale_old + acc_block * scale_new
+        m = m_new
+        trace.append((m, l, np.array(acc, copy=True)))
+    return acc / l, m, l, trace
+
+
+def online_softmax_row_runningmax(scores, values, block: int):
+    """One query row, tiled, with exponentials taken relative to the updated
+    running max (page "FlashAttention: The GPU Memory Hack That Changed
+    Everything", section "The Tiling Strategy": l = l*exp(m - m_new) +
+    sum exp(S - m_new); O = O*exp(m - m_new) + exp(S - m_new) V; final O/l).
+    Returns (O, m, l).
+    """
+    s = np.asarray(scores, dtype=np.float64)
+    vals = np.asarray(values, dtype=np.float64)
+    n = s.shape[0]
+    m = -np.inf
+    l = 0.0
+    acc = np.zeros(vals.shape[1:], dtype=np.float64)
+    for start in range(0, n, block):
+        sb = s[start:start + block]
+        vb = vals[start:start + block]
+        m_new = max(m, np.max(sb))
+        alpha = np.exp(m - m_new)
+        p = np.exp(sb - m_new)
+        l = l * alpha + np.sum(p)
+        acc = acc * alpha + np.tensordot(p, vb, axes=(0, 0))
+        m = m_new
+    return acc / l, m, l
+
+
+def tiled_attention_fp64(q, k, v, causal: bool, scale: float, block_q: int,
+                         block_k: int):
+    """Whole-matrix tiled forward for one (N, d) head: Q blocks outer, K/V
+    blocks inner, running (m, l, acc) per row (page "FlashAttention: The GPU
+    Memory Hack That Changed Everything", section "The Tiling Strategy").
+    Causal K/V blocks that lie entirely above the diagonal are skipped, and
+    partially masked entries are -inf.  Self-test companion only.
+    Returns (O (N, d), LSE (N,)).
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    N, d = q.shape
+    O = np.empty((N, d))
+    LSE = np.empty(N)
+    for i0 in range(0, N, block_q):
+        i1 = min(N, i0 + block_q)
+        qi = q[i0:i1]
+        m = np.full(i1 - i0, -np.inf)
+        l = np.zeros(i1 - i0)
+        acc = np.zeros((i1 - i0, d))
+        for j0 in range(0, N, block_k):
+            if causal and j0 > i1 - 1:
+                break                                   # block fully above the diagonal
+            j1 = min(N, j0 + block_k)
+            Sij = scale * (qi @ k[j0:j1].T)
+            if causal:
+                ii = np.arange(i0, i1)[:, None]
+                jj = np.arange(j0, j1)[None, :]
+                Sij = np.where(jj <= ii, Sij, -np.inf)
+            m_new = np.maximum(m, Sij.max(axis=1))
+            alpha = np.exp(m - m_new)
+            p = np.exp(Sij - m_new[:, None])
+            l = l * alpha + p.sum(axis=1)
+            acc = acc * alpha[:, None] + p @ v[j0:j1]
+            m = m_new
+        O[i0:i1] = acc / l[:, None]
+        LSE[i0:i1] = m + np.log(l)
+    return O, LSE

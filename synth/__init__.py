@@ -1,0 +1,94 @@
+"""Seeded synthetic inputs shared by the tests, the oracle checks and bench.py.
+
+This module draws random numbers and casts them to bfloat16; it holds none of
+the attention arithmetic.  The pages measure on no dataset: "BERT" and "GPT-2"
+in the page "FlashAttention: The GPU Memory Hack That Changed Everything"
+(section "Speed Improvements") supply only sequence lengths, and its
+"Try It Yourself" script draws ``torch.randn`` Q, K, V of shape
+(batch, heads, seq_len, head_dim).  The workloads below follow that recipe.
+
+Recipe (one CPU ``torch.Generator`` per workload, seed 1220 + workload index):
+draw Q, K, V in that order as float32 standard normals of shape (B, H, N, d),
+multiply Q and K by ``qk_std`` (3.0 for the peaked long-context workload, so
+the scaled scores have standard deviation 9), then round to bfloat16
+(round-to-nearest-even, torch's cast).  Both the CUDA path and the oracle
+consume these exact bf16 tensors.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    index: int
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    qk_std: float = 1.0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def seed(self) -> int:
+        return 1220 + self.index
+
+    @property
+    def flops(self) -> float:
+        """4*B*H*N^2*d, halved when causal (the path's FLOP convention)."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    @property
+    def algorithmic_bytes(self) -> int:
+        """Q, K, V read once and O written once (bf16) plus the fp32 LSE."""
+        elems = self.B * self.H * self.N * self.d
+        return 4 * elems * 2 + self.B * self.H * self.N * 4
+
+    def describe(self) -> str:
+        return (f"{self.name}: B={self.B} H={self.H} N={self.N} d={self.d} "
+                f"{'causal' if self.causal else 'non-causal'}")
+
+
+WORKLOADS = [
+    Workload(1, "toy_single_head", 1, 1, 256, 64, False),
+    Workload(2, "bert_base_encoder", 8, 12, 512, 64, False),
+    Workload(3, "gpt2_small_decoder", 8, 12, 1024, 64, True),
+    Workload(4, "long_context_causal", 2, 32, 8192, 128, True),
+    Workload(5, "very_long_peaked_causal", 1, 16, 32768, 128, True, qk_std=3.0),
+]
+
+
+def workload(index_or_name) -> Workload:
+    for w in WORKLOADS:
+        if w.index == index_or_name or w.name == index_or_name:
+            return w
+    raise KeyError(index_or_name)
+
+
+def draw_qkv(B: int, H: int, N: int, d: int, seed: int, qk_std: float = 1.0):
+    """Seeded bf16 Q, K, V on the CPU, shape (B, H, N, d), contiguous."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    shape = (B, H, N, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    if qk_std != 1.0:
+        q.mul_(qk_std)
+        k.mul_(qk_std)
+    return (q.to(torch.bfloat16).contiguous(), k.to(torch.bfloat16).contiguous(),
+            v.to(torch.bfloat16).contiguous())
+
+
+def workload_qkv(w: Workload):
+    return draw_qkv(w.B, w.H, w.N, w.d, w.seed, w.qk_std)
