@@ -1,0 +1,14 @@
+"""exact_attention_122_b200 -- exact attention forward on B200 (sm_100a).
+
+The computation lives in the CUDA library libfa_b200.so behind the C ABI of
+include/fa.h; this module only marshals arguments to it (torch supplies
+device memory and streams).  There is no CPU fallback: if the library is
+missing, importing the binding raises.
+"""
+
+from ._binding import (  # noqa: F401
+    FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_MISALIGNED, FA_ERR_LAUNCH,
+    FA_ERR_TIMEOUT, FA_ERR_NO_DEVICE, EXPORTED_SYMBOLS,
+    FaError, library, library_path, status_string, version,
+    fa_fwd, fa_fwd_raw, fa_fwd_debug_raw, device_status,
+)

@@ -1,0 +1,126 @@
+"""ctypes binding of libfa_b200.so (include/fa.h).  Argument marshalling only."""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_MISALIGNED = 3
+FA_ERR_LAUNCH = 4
+FA_ERR_TIMEOUT = 5
+FA_ERR_NO_DEVICE = 6
+
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_debug", "fa_get_device_status", "fa_status_string",
+                    "fa_last_cuda_error", "fa_version")
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libfa_b200.so")
+
+
+def library() -> ctypes.CDLL:
+    """Load libfa_b200.so once; raise if it has not been built."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m exact_attention_122_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    vp, i, f, u = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint
+    fwd_args = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+    lib.fa_fwd.argtypes = fwd_args
+    lib.fa_fwd.restype = i
+    lib.fa_fwd_debug.argtypes = fwd_args + [u, i]
+    lib.fa_fwd_debug.restype = i
+    lib.fa_get_device_status.argtypes = [vp, ctypes.POINTER(u)]
+    lib.fa_get_device_status.restype = i
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_last_cuda_error.argtypes = []
+    lib.fa_last_cuda_error.restype = i
+    lib.fa_version.argtypes = []
+    lib.fa_version.restype = i
+    _LIB = lib
+    return lib
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str = "fa_fwd"):
+        self.status = status
+        name = status_string(status)
+        extra = ""
+        if status in (FA_ERR_LAUNCH, FA_ERR_NO_DEVICE):
+            extra = f" (cudaError {library().fa_last_cuda_error()})"
+        super().__init__(f"{what} failed: {name}{extra}")
+
+
+def status_string(status: int) -> str:
+    return library().fa_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return library().fa_version()
+
+
+def fa_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int,
+               N: int, d: int, causal: int, scale: float, stream_ptr: int) -> int:
+    """Direct call of the C entry point; returns the fa_status code."""
+    return library().fa_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal, scale,
+                            stream_ptr)
+
+
+def fa_fwd_debug_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal, scale, stream_ptr,
+                     watchdog_ms: int, inject: int) -> int:
+    return library().fa_fwd_debug(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal, scale,
+                                  stream_ptr, watchdog_ms, inject)
+
+
+def device_status(stream_ptr: int = 0):
+    """(status, raw word) of the kernel watchdog; synchronises the stream."""
+    word = ctypes.c_uint(0)
+    st = library().fa_get_device_status(stream_ptr, ctypes.byref(word))
+    return st, word.value
+
+
+def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+           stream=None):
+    """O, LSE = exact attention forward of bf16 (B, H, N, d) CUDA tensors.
+
+    ``out`` (bf16, same shape) and ``lse`` (float32, (B, H, N)) are allocated
+    with torch when not given.  Runs asynchronously on ``stream`` (default:
+    the current torch stream of q's device).
+    """
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor of shape (B, H, N, d)")
+    if k.shape != q.shape or v.shape != q.shape or k.device != q.device or v.device != q.device:
+        raise ValueError("q, k, v must share shape and device")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if not (out.is_cuda and out.dtype == torch.bfloat16 and out.shape == q.shape and out.is_contiguous()):
+        raise ValueError("out must be a contiguous bf16 CUDA tensor shaped like q")
+    if not (lse.is_cuda and lse.dtype == torch.float32 and tuple(lse.shape) == (B, H, N) and lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 CUDA tensor of shape (B, H, N)")
+    with torch.cuda.device(q.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        st = fa_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                        B, H, N, d, 1 if causal else 0, float(scale), s.cuda_stream)
+    if st != FA_OK:
+        raise FaError(st)
+    return out, lse

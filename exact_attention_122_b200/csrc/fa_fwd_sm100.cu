@@ -1,0 +1,910 @@
+// fa_fwd_sm100.cu -- exact attention forward for B200 (sm_100a).
+//
+// Computes, per (batch, head), O = softmax(scale * Q K^T [+ causal mask]) V
+// and the per-row log-sum-exp, tile by tile with the online-softmax
+// recurrence, so the N x N score matrix never leaves the SM:
+//   * page "Flash attention optimization", section "Attention is not slow
+//     because of arithmetic" (the definition) and "The fix: tile the
+//     computation, never materialize the full matrix" (running max m,
+//     running sum l, rescaled accumulator, final acc / l);
+//   * page "FlashAttention: The GPU Memory Hack That Changed Everything",
+//     section "The Tiling Strategy" (Q blocks outer, K/V blocks inner, the
+//     exponent taken relative to the updated running max) and
+//     "FlashAttention-2: Even Faster" (work split over the sequence as well
+//     as batch x heads; fewer non-matmul operations);
+//   * same page, "FlashAttention-3: Hopper Architecture" (asynchronous
+//     copies, warp specialisation), re-done for sm_100a with TMA, mbarriers,
+//     tcgen05 MMAs and tensor memory (TMEM).
+//
+// Kernel organisation (one persistent CTA per SM, 384 threads):
+//   warps 0-3  softmax warpgroup 0: rows 0..127 of the current 256-row unit
+//   warps 4-7  softmax warpgroup 1: rows 128..255
+//   warp  8    MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j
+//   warp  9    TMA producer (one thread): Q_0, Q_1 per unit, then K_j, V_j
+//              through an NS-stage shared-memory ring
+//   warps 10-11 idle (they complete the third warpgroup)
+// The third warpgroup gives registers to the softmax warpgroups with
+// setmaxnreg (REGS_SOFTMAX / REGS_OTHER below).
+// Each softmax thread owns one query row (TMEM lane == row), so the row max
+// and row sum are in-thread.  S_t (fp32, 128 columns) and O_t (fp32, d
+// columns) live in TMEM; P_t is written back as bf16 over the first 64
+// columns of S_t and read from TMEM by the PV MMA.  The two warpgroups
+// alternate with the single MMA issuer, so the tensor core works on one
+// sub-tile while the other sub-tile's exponentials run.
+//
+// Every mbarrier wait is bounded by a %globaltimer watchdog.  A wait that
+// runs out records FA_ERR_TIMEOUT in g_fa_status, raises a CTA-wide abort
+// flag so every role leaves its loop, drains its own TMA copies and MMAs
+// (again bounded), frees TMEM and returns.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+
+namespace fa {
+
+// ---------------------------------------------------------------------------
+// Tile geometry
+// ---------------------------------------------------------------------------
+constexpr int BM = 128;            // query rows per sub-tile (= TMEM lanes)
+constexpr int BN = 128;            // keys per K/V tile
+constexpr int UNIT_ROWS = 2 * BM;  // query rows per work unit (two sub-tiles)
+constexpr int NUM_THREADS = 384;
+constexpr int MMA_WARP = 8;
+constexpr int TMA_WARP = 9;
+// Register split.  The launch gives every thread REGS_LAUNCH registers
+// (65536 / 384, rounded down to 8 and to the sub-partition share: 168).
+// Warpgroup 2 drops to REGS_OTHER once at the start and never rises again;
+// warpgroups 0 and 1 rise to REGS_SOFTMAX.  The sum must not exceed the
+// launch total or setmaxnreg.inc never returns.
+constexpr int REGS_LAUNCH = 168;
+constexpr int REGS_SOFTMAX = 208;
+constexpr int REGS_OTHER = 80;
+static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER <= NUM_THREADS * REGS_LAUNCH,
+              "register split exceeds the launch allocation");
+constexpr int SW_COLS = 64;        // bf16 elements per 128-byte swizzled row
+
+enum : uint32_t {
+    ROLE_SOFTMAX = 1u, ROLE_MMA = 2u, ROLE_PRODUCER = 3u, ROLE_DRAIN = 4u
+};
+
+template <int D, int NS>
+struct Layout {
+    static constexpr int Q_BYTES = BM * D * 2;       // one sub-tile of Q
+    static constexpr int KV_BYTES = BN * D * 2;      // one K or V tile
+    static constexpr int HALF_BYTES = BM * SW_COLS * 2;  // one 64-column slab (16 KiB)
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_KV = 2 * Q_BYTES;
+    static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
+    // barrier slots
+    static constexpr int B_KV_FULL = 0;
+    static constexpr int B_KV_EMPTY = NS;
+    static constexpr int B_Q_FULL = 2 * NS;
+    static constexpr int B_Q_EMPTY = 2 * NS + 1;
+    static constexpr int B_S_FULL = 2 * NS + 2;      // [2]
+    static constexpr int B_P_FULL = 2 * NS + 4;      // [2]
+    static constexpr int B_O_FULL = 2 * NS + 6;      // [2]
+    static constexpr int B_O_EMPTY = 2 * NS + 8;     // [2]
+    static constexpr int B_DRAIN = 2 * NS + 10;
+    static constexpr int NUM_BARS = 2 * NS + 11;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem base, abort flag
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int ALLOC = BYTES + 1024;       // slack to align the base to 1 KiB
+    // TMEM columns
+    static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+    static constexpr uint32_t TM_COLS = 512;
+    static_assert(ALLOC <= 227 * 1024, "shared memory budget");
+    static_assert(BYTES > 116 * 1024, "one CTA per SM keeps TMEM allocation uncontended");
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ unsigned int g_fa_status;  // 0 = fine; else (FA_ERR_TIMEOUT << 24) | role << 20 | unit
+
+struct Watchdog {
+    volatile int* abort_flag;
+    uint64_t limit_ns;
+};
+
+// Waits for the phase of `bar` with the given parity to complete.  Returns
+// false if the CTA is aborting or this wait ran past the watchdog limit (in
+// which case it records the timeout and raises the abort flag).
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Watchdog wd,
+                                        uint32_t role, uint32_t unit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*wd.abort_flag) return false;
+        if (global_timer_ns() - t0 > wd.limit_ns) {
+            atomicCAS(&g_fa_status, 0u,
+                      (uint32_t(FA_ERR_TIMEOUT) << 24) | (role << 20) | (unit & 0xFFFFFu));
+            *wd.abort_flag = 1;
+            __threadfence_block();
+            return false;
+        }
+    }
+}
+
+// TMA: 3-D tiled load (d offset, row, batch*head) into shared memory,
+// completing `bytes` on the mbarrier.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// ---- tcgen05 (5th-generation tensor core, tensor memory) ----
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrive once on `bar` when every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+}
+// D(tmem) (+)= A(smem desc) * B(smem desc)
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D(tmem) (+)= A(tmem) * B(smem desc)
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane, waited on inside
+// the same asm statement so no register is read before it is valid.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+template <int R>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+
+// Barrier 0 over all NUM_THREADS threads, usable from different branches.
+__device__ __forceinline__ void cta_sync() {
+    asm volatile("bar.sync 0, %0;" ::"n"(NUM_THREADS) : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ---- UMMA descriptors ----
+// Shared-memory matrix descriptor, 128-byte swizzle (the layout TMA writes
+// with CU_TENSOR_MAP_SWIZZLE_128B): start address, leading and stride byte
+// offsets (16-byte units), descriptor version 1, swizzle mode 2.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+    d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+    d |= uint64_t(1) << 46;
+    d |= uint64_t(2) << 61;
+    return d;
+}
+
+// Instruction descriptor for kind::f16: fp32 accumulator, bf16 A and B,
+// A K-major, B K-major or MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// Work decomposition: units of 256 query rows of one (batch, head).  Unit u
+// is (level, bh) with level = u / BH; for causal masking the level counts
+// down from the last (longest) row block so the longest units go first.
+// ---------------------------------------------------------------------------
+struct Unit {
+    int bh, r0, nb0, nb1;  // first row, K/V tile counts of sub-tiles 0 and 1
+};
+
+__device__ __forceinline__ Unit decode_unit(int u, int BH, int N, int causal) {
+    const int nq2 = (N + UNIT_ROWS - 1) / UNIT_ROWS;
+    const int nkb = (N + BN - 1) / BN;
+    const int level = u / BH;
+    Unit w;
+    w.bh = u - level * BH;
+    const int qb2 = causal ? (nq2 - 1 - level) : level;
+    w.r0 = qb2 * UNIT_ROWS;
+    if (causal) {
+        w.nb0 = min(w.r0 / BN + 1, nkb);
+        w.nb1 = min(w.r0 / BN + 2, nkb);
+    } else {
+        w.nb0 = nkb;
+        w.nb1 = nkb;
+    }
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+template <int D, int NS>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ Og,
+                  float* __restrict__ LSEg, int BH, int N, int causal, float scale_log2,
+                  unsigned long long watchdog_ns, int inject) {
+    using L = Layout<D, NS>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t sQ = sbase + L::OFF_Q;
+    const uint32_t sKV = sbase + L::OFF_KV;
+    const uint32_t sBar = sbase + L::OFF_BAR;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nq2 = (N + UNIT_ROWS - 1) / UNIT_ROWS;
+    const int num_units = nq2 * BH;
+    const int nkb = (N + BN - 1) / BN;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(L::B_KV_FULL + s), 1);
+            mbar_init(bar(L::B_KV_EMPTY + s), 1);
+        }
+        mbar_init(bar(L::B_Q_FULL), 1);
+        mbar_init(bar(L::B_Q_EMPTY), 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar(L::B_S_FULL + t), 1);
+            mbar_init(bar(L::B_P_FULL + t), BM);
+            mbar_init(bar(L::B_O_FULL + t), 1);
+            mbar_init(bar(L::B_O_EMPTY + t), BM);
+        }
+        mbar_init(bar(L::B_DRAIN), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), L::TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Watchdog wd{abort_flag, watchdog_ns};
+
+    // Each role's code sits inside the branch that set its register budget,
+    // so ptxas allocates it against that budget.
+    if (warp >= 8) {
+    regs_dec<REGS_OTHER>();
+    if (warp >= 10) {
+        // idle warps of the third warpgroup
+    } else if (warp == TMA_WARP) {
+        // ------------------------------------------------------------------
+        // Producer: Q_0/Q_1 per unit, then K_0, V_0, K_1, V_1, ... through
+        // the ring.  fills counts ring loads over the CTA's lifetime.
+        // ------------------------------------------------------------------
+        if (lane == 0) {
+            uint32_t fills = 0, units = 0, q_issued = 0;
+            uint32_t stage_fill[NS];        // last fill index issued into each stage, +1
+            for (int s = 0; s < NS; ++s) stage_fill[s] = 0;
+            bool ok = true;
+            bool skipped = false;
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++units) {
+                const Unit w = decode_unit(u, BH, N, causal);
+                if (!wait_phase(bar(L::B_Q_EMPTY), (units & 1u) ^ 1u, wd, ROLE_PRODUCER, u)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(bar(L::B_Q_FULL), 2 * L::Q_BYTES);
+                for (int t = 0; t < 2; ++t)
+                    for (int h = 0; h < D / SW_COLS; ++h)
+                        tma_load_3d(sQ + t * L::Q_BYTES + h * L::HALF_BYTES, &tmQ, h * SW_COLS,
+                                    w.r0 + t * BM, w.bh, bar(L::B_Q_FULL));
+                ++q_issued;
+                for (int j = 0; j < w.nb1 && ok; ++j) {
+                    for (int kind = 0; kind < 2; ++kind) {
+                        const uint32_t s = fills % NS;
+                        const uint32_t ph = (fills / NS) & 1u;
+                        if (!wait_phase(bar(L::B_KV_EMPTY + s), ph ^ 1u, wd, ROLE_PRODUCER, u)) {
+                            ok = false;
+                            break;
+                        }
+                        const bool skip = inject == 1 && !skipped && blockIdx.x == 0;
+                        if (skip) {
+                            skipped = true;  // fault injection: this copy is never issued
+                        } else {
+                            mbar_arrive_expect_tx(bar(L::B_KV_FULL + s), L::KV_BYTES);
+                            const CUtensorMap* map = kind == 0 ? &tmK : &tmV;
+                            for (int h = 0; h < D / SW_COLS; ++h)
+                                tma_load_3d(sKV + s * L::KV_BYTES + h * L::HALF_BYTES, map,
+                                            h * SW_COLS, j * BN, w.bh, bar(L::B_KV_FULL + s));
+                            stage_fill[s] = fills + 1;
+                        }
+                        ++fills;
+                    }
+                }
+            }
+            if (!ok) {
+                // Drain: wait (bounded) for every copy this thread issued.
+                Watchdog dwd{abort_flag, wd.limit_ns};
+                volatile int never = 0;
+                dwd.abort_flag = &never;
+                for (int s = 0; s < NS; ++s)
+                    if (stage_fill[s] != 0)
+                        wait_phase(bar(L::B_KV_FULL + s), ((stage_fill[s] - 1) / NS) & 1u, dwd,
+                                   ROLE_DRAIN, 0);
+                if (q_issued > 0)
+                    wait_phase(bar(L::B_Q_FULL), (q_issued - 1) & 1u, dwd, ROLE_DRAIN, 0);
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        // ------------------------------------------------------------------
+        // MMA issuer.  Per unit: S_0 = Q_0 K_0^T, S_1 = Q_1 K_0^T; then per
+        // K/V tile j: O_0 += P_0 V_j, S_0 = Q_0 K_{j+1}^T, O_1 += P_1 V_j,
+        // S_1 = Q_1 K_{j+1}^T.  tcgen05 MMAs from one thread execute in
+        // issue order, so P_t (aliasing S_t) is consumed before the next S_t
+        // overwrites it, and a commit after S_t also covers the PV before it.
+        // ------------------------------------------------------------------
+        if (lane == 0) {
+            constexpr uint32_t ID_S = idesc_bf16(BM, BN, false);
+            constexpr uint32_t ID_PV = idesc_bf16(BM, D, true);
+            uint32_t cons = 0, units = 0, pcnt0 = 0, pcnt1 = 0;
+            bool ok = true;
+            bool issued = false;
+            auto issue_s = [&](int t, uint32_t kstage) {
+                const uint32_t dS = tmem + (t ? L::TM_S1 : L::TM_S0);
+                const uint32_t qa = sQ + t * L::Q_BYTES;
+                const uint32_t ka = sKV + kstage * L::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    // K-major operands: 16 bf16 of d per MMA; 32 bytes inside a
+                    // 128-byte swizzled row, 64-column slabs 16 KiB apart.
+                    const uint32_t off = (kk / 4) * L::HALF_BYTES + (kk % 4) * 32;
+                    mma_ss(dS, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+                           ID_S, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int t, uint32_t vstage, bool first) {
+                const uint32_t dO = tmem + (t ? L::TM_O1 : L::TM_O0);
+                const uint32_t aP = tmem + (t ? L::TM_S1 : L::TM_S0);
+                const uint32_t va = sKV + vstage * L::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    // A = P from TMEM (16 keys = 8 columns of bf16 pairs); B = V,
+                    // MN-major: 16 key rows of 128 bytes per step, d slabs 16 KiB
+                    // apart (leading byte offset), 8-row groups 1 KiB apart.
+                    mma_ts(dO, aP + kk * 8, sdesc_sw128(va + kk * 16 * 128, L::HALF_BYTES, 1024),
+                           ID_PV, (first && kk == 0) ? 0u : 1u);
+                }
+            };
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++units) {
+                const Unit w = decode_unit(u, BH, N, causal);
+                if (!wait_phase(bar(L::B_Q_FULL), units & 1u, wd, ROLE_MMA, u)) { ok = false; break; }
+                uint32_t sK = cons % NS;
+                if (!wait_phase(bar(L::B_KV_FULL + sK), (cons / NS) & 1u, wd, ROLE_MMA, u)) {
+                    ok = false;
+                    break;
+                }
+                ++cons;
+                issue_s(0, sK);
+                tc_commit(bar(L::B_S_FULL + 0));
+                issue_s(1, sK);
+                tc_commit(bar(L::B_S_FULL + 1));
+                tc_commit(bar(L::B_KV_EMPTY + sK));
+                issued = true;
+                if (w.nb1 == 1) tc_commit(bar(L::B_Q_EMPTY));
+                for (int j = 0; j < w.nb1; ++j) {
+                    const uint32_t sV = cons % NS;
+                    if (!wait_phase(bar(L::B_KV_FULL + sV), (cons / NS) & 1u, wd, ROLE_MMA, u)) {
+                        ok = false;
+                        break;
+                    }
+                    ++cons;
+                    const bool next = j + 1 < w.nb1;
+                    if (next) {
+                        sK = cons % NS;
+                        if (!wait_phase(bar(L::B_KV_FULL + sK), (cons / NS) & 1u, wd, ROLE_MMA, u)) {
+                            ok = false;
+                            break;
+                        }
+                        ++cons;
+                    }
+                    if (j < w.nb0) {
+                        if (j == 0 && !wait_phase(bar(L::B_O_EMPTY + 0), (units & 1u) ^ 1u, wd,
+                                                  ROLE_MMA, u)) {
+                            ok = false;
+                            break;
+                        }
+                        if (!wait_phase(bar(L::B_P_FULL + 0), pcnt0 & 1u, wd, ROLE_MMA, u)) {
+                            ok = false;
+                            break;
+                        }
+                        ++pcnt0;
+                        tc_fence_after();
+                        issue_pv(0, sV, j == 0);
+                        if (j + 1 < w.nb0) {
+                            issue_s(0, sK);
+                            tc_commit(bar(L::B_S_FULL + 0));
+                        }
+                        if (j == w.nb0 - 1) tc_commit(bar(L::B_O_FULL + 0));
+                    }
+                    if (j == 0 && !wait_phase(bar(L::B_O_EMPTY + 1), (units & 1u) ^ 1u, wd, ROLE_MMA, u)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!wait_phase(bar(L::B_P_FULL + 1), pcnt1 & 1u, wd, ROLE_MMA, u)) {
+                        ok = false;
+                        break;
+                    }
+                    ++pcnt1;
+                    tc_fence_after();
+                    issue_pv(1, sV, j == 0);
+                    if (next) {
+                        issue_s(1, sK);
+                        tc_commit(bar(L::B_S_FULL + 1));
+                    }
+                    tc_commit(bar(L::B_KV_EMPTY + sV));
+                    if (next) tc_commit(bar(L::B_KV_EMPTY + sK));
+                    if (next && j + 1 == w.nb1 - 1) tc_commit(bar(L::B_Q_EMPTY));
+                    if (j == w.nb1 - 1) tc_commit(bar(L::B_O_FULL + 1));
+                }
+            }
+            if (issued) {
+                // Every MMA this thread issued must finish before TMEM is
+                // freed; on the normal path the softmax warps have already
+                // waited for the last O commit, so this returns at once.
+                Watchdog dwd{abort_flag, wd.limit_ns};
+                volatile int never = 0;
+                dwd.abort_flag = &never;
+                tc_commit(bar(L::B_DRAIN));
+                wait_phase(bar(L::B_DRAIN), 0, dwd, ROLE_DRAIN, 0);
+            }
+        }
+        __syncwarp();
+    }
+    // Teardown of warpgroup 2: after every thread of the CTA is done with
+    // TMEM, the allocating warp frees it.
+    tc_fence_before();
+    cta_sync();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TM_COLS);
+    }
+    } else {
+        // ------------------------------------------------------------------
+        // Softmax warpgroups.  Thread = query row; TMEM lane = row.
+        // ------------------------------------------------------------------
+        regs_inc<REGS_SOFTMAX>();
+        const int t = warp >> 2;                     // sub-tile 0 or 1
+        const int wr = (warp & 3) * 32 + lane;       // row within the sub-tile
+        const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + (t == 0 ? L::TM_S0 : L::TM_S1);
+        const uint32_t tO = tmem + lane_base + (t == 0 ? L::TM_O0 : L::TM_O1);
+        uint32_t scnt = 0, ocnt = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const Unit w = decode_unit(u, BH, N, causal);
+            const int a = w.r0 + t * BM;             // first row of this sub-tile
+            const int row = a + wr;
+            const int nb = t == 0 ? w.nb0 : w.nb1;
+            float m = -INFINITY;                     // running max, log2 units
+            float l = 0.f;                           // running sum of exponentials
+            for (int j = 0; j < nb; ++j) {
+                bool got = wait_phase(bar(L::B_S_FULL + t), scnt & 1u, wd, ROLE_SOFTMAX, u);
+                ++scnt;
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
+                float s[BN];
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + c * 32, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+                }
+                // Mask: keys beyond N on the last tile; keys above the
+                // diagonal on a sub-tile's diagonal tile.
+                const bool tail = (j == nkb - 1) && (N % BN != 0);
+                const bool diag = causal && (j == a / BN);
+                if (tail || diag) {
+                    const int lim_tail = N - j * BN;           // key c allowed iff c < lim_tail
+                    const int lim_diag = row - j * BN;         // key c allowed iff c <= lim_diag
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) {
+                        const bool bad = (c >= lim_tail) || (causal && c > lim_diag);
+                        s[c] = bad ? -INFINITY : s[c];
+                    }
+                }
+                float mx = s[0];
+#pragma unroll
+                for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+                const float m_new = fmaxf(m, mx * scale_log2);
+                const float alpha = ex2(m - m_new);          // 0 on the first tile (m = -inf)
+                if (j > 0 && __any_sync(0xffffffffu, m_new > m)) {
+                    // Rescale this warp's rows of O (the PV of tile j-1 is
+                    // complete: its commit preceded the S_t commit above).
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(tO + c * 32, r);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st32(tO + c * 32, r);
+                    }
+                }
+                l *= alpha;
+                m = m_new;
+                const float neg_m = -m;
+                float rowsum = 0.f;
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = ex2(fmaf(s[c * 32 + 2 * i], scale_log2, neg_m));
+                        const float p1 = ex2(fmaf(s[c * 32 + 2 * i + 1], scale_log2, neg_m));
+                        rowsum += p0 + p1;
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + c * 16, pk);              // P (bf16) over S columns [0, 64)
+                }
+                l += rowsum;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(L::B_P_FULL + t));
+            }
+            if (!ok) break;
+            // Epilogue: O / l -> bf16 -> global; LSE.
+            bool got = wait_phase(bar(L::B_O_FULL + t), ocnt & 1u, wd, ROLE_SOFTMAX, u);
+            ++ocnt;
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+            const float inv_l = 1.f / l;
+            const bool store = row < N;
+            __nv_bfloat16* orow = Og + (size_t(w.bh) * N + (store ? row : 0)) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tO + c * 32, r);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
+                                        __uint_as_float(r[2 * i + 1]) * inv_l);
+                if (store) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                }
+            }
+            if (store) LSEg[size_t(w.bh) * N + row] = (m + log2f(l)) * 0.69314718055994530942f;
+            tc_fence_before();
+            mbar_arrive(bar(L::B_O_EMPTY + t));
+        }
+        tc_fence_before();
+        cta_sync();
+    }
+    // The two branches meet only at kernel exit: no code runs after them,
+    // so neither warpgroup has to give its register budget back.
+}
+
+}  // namespace fa
+
+// ===========================================================================
+// Host side: validation, tensor maps, launch.
+// ===========================================================================
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+thread_local int t_last_cuda_error = 0;
+
+constexpr int MAX_DEVICES = 64;
+struct DeviceInfo {
+    std::once_flag once;
+    int ok = 0;
+    int sm_count = 0;
+    int cc_major = 0, cc_minor = 0;
+};
+DeviceInfo g_dev[MAX_DEVICES];
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+template <int D, int NS>
+struct Instance {
+    static std::once_flag once[MAX_DEVICES];
+    static cudaError_t attr_err[MAX_DEVICES];
+    static int regs[MAX_DEVICES];
+};
+template <int D, int NS>
+std::once_flag Instance<D, NS>::once[MAX_DEVICES];
+template <int D, int NS>
+cudaError_t Instance<D, NS>::attr_err[MAX_DEVICES];
+template <int D, int NS>
+int Instance<D, NS>::regs[MAX_DEVICES];
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+fa_status encode_map(CUtensorMap* map, const void* base, int d, int N, long long BH) {
+    const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+    const cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(d) * 2 * cuuint64_t(N)};
+    const cuuint32_t box[3] = {cuuint32_t(fa::SW_COLS), cuuint32_t(fa::BM), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+template <int D, int NS>
+fa_status launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int causal, float scale, cudaStream_t stream, int dev,
+                 unsigned long long watchdog_ns, int inject) {
+    using L = fa::Layout<D, NS>;
+    auto kern = fa::fa_fwd_kernel<D, NS>;
+    std::call_once(Instance<D, NS>::once[dev], [&] {
+        Instance<D, NS>::attr_err[dev] =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+        cudaFuncAttributes fa_attr;
+        if (Instance<D, NS>::attr_err[dev] == cudaSuccess &&
+            cudaFuncGetAttributes(&fa_attr, kern) == cudaSuccess)
+            Instance<D, NS>::regs[dev] = fa_attr.numRegs;
+    });
+    if (Instance<D, NS>::attr_err[dev] != cudaSuccess) {
+        t_last_cuda_error = int(Instance<D, NS>::attr_err[dev]);
+        return FA_ERR_LAUNCH;
+    }
+    // The setmaxnreg split was sized for REGS_LAUNCH registers per thread;
+    // with any other launch allocation setmaxnreg.inc could wait forever,
+    // so such a build is refused rather than launched.
+    if (Instance<D, NS>::regs[dev] != fa::REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
+    const long long BH = (long long)B * H;
+    CUtensorMap mq, mk, mv;
+    if (encode_map(&mq, q, D, N, BH) != FA_OK || encode_map(&mk, k, D, N, BH) != FA_OK ||
+        encode_map(&mv, v, D, N, BH) != FA_OK)
+        return FA_ERR_UNSUPPORTED;
+    const long long nq2 = (N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+    const long long units = nq2 * BH;
+    const int grid = int(units < g_dev[dev].sm_count ? units : g_dev[dev].sm_count);
+    const float scale_log2 = scale * 1.4426950408889634f;
+    kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o),
+                                                     lse, int(BH), N, causal, scale_log2,
+                                                     watchdog_ns, inject);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        t_last_cuda_error = int(e);
+        return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int N, int d, int causal, float scale, void* stream, unsigned watchdog_ms,
+                   int inject) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (inject != 0 && inject != 1) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0x7fffffffLL || N > (1 << 30)) return FA_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return FA_ERR_MISALIGNED;
+
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
+        t_last_cuda_error = int(e);
+        return FA_ERR_NO_DEVICE;
+    }
+    DeviceInfo& di = g_dev[dev];
+    std::call_once(di.once, [&] {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return;
+        di.sm_count = prop.multiProcessorCount;
+        di.cc_major = prop.major;
+        di.cc_minor = prop.minor;
+        di.ok = 1;
+    });
+    if (!di.ok) return FA_ERR_NO_DEVICE;
+    if (di.cc_major != 10 || di.cc_minor != 0) return FA_ERR_UNSUPPORTED;
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) ==
+                cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    if (!g_encode) return FA_ERR_NO_DEVICE;
+
+    const unsigned long long wd_ns = (watchdog_ms ? watchdog_ms : 4000u) * 1000000ull;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d == 64) return launch<64, 8>(q, k, v, o, lse, B, H, N, causal, scale, s, dev, wd_ns, inject);
+    return launch<128, 4>(q, k, v, o, lse, B, H, N, causal, scale, s, dev, wd_ns, inject);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, int causal, float scale, void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, stream, 0, 0);
+}
+
+fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int N, int d, int causal, float scale, void* stream,
+                       unsigned watchdog_ms, int inject) {
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, stream, watchdog_ms, inject);
+}
+
+fa_status fa_get_device_status(void* stream, unsigned* detail) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned word = 0;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&word, fa::g_fa_status, sizeof(word));
+    const unsigned zero = 0;
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) {
+        t_last_cuda_error = int(e);
+        return e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver ? FA_ERR_NO_DEVICE
+                                                                           : FA_ERR_LAUNCH;
+    }
+    if (detail) *detail = word;
+    return word == 0 ? FA_OK : FA_ERR_TIMEOUT;
+}
+
+const char* fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+        case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+        case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH";
+        case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+        case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE";
+        default: return "FA_ERR_UNKNOWN";
+    }
+}
+
+int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

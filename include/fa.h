@@ -1,0 +1,118 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention forward library
+ *         (libfa_b200.so, built from exact_attention_122_b200/csrc/).
+ *
+ * The operation (page "Flash attention optimization", section "Attention is
+ * not slow because of arithmetic"): for every batch b and head h, with Q, K,
+ * V in R^{N x d},
+ *
+ *     S = scale * Q K^T,   P = softmax(S) row-wise,   O = P V,
+ *
+ * computed tile by tile with the online-softmax recurrence (same page, "The
+ * fix: tile the computation, never materialize the full matrix"; page
+ * "FlashAttention: The GPU Memory Hack That Changed Everything", "The Tiling
+ * Strategy"), so no N x N matrix ever reaches device memory.  With causal
+ * masking (that page's is_causal=True, "Integration: It's Everywhere") key j
+ * is allowed for query i iff j <= i.  The result is exact up to rounding
+ * order; O is rounded to bf16 once at the end.
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers named q, k, v, o, lse are DEVICE pointers owned by the caller.
+ *    The library never allocates, frees or retains them.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *    the legacy default stream) and the call returns without synchronising.
+ *    Results are valid once the caller has synchronised that stream.
+ *  - Arguments are validated before anything is enqueued; an invalid call
+ *    returns an error status and has no side effect.
+ *  - Calls are thread-safe.  One call per stream at a time may run on a
+ *    device; concurrent calls on different streams are independent.
+ *  - Inputs holding NaN or Inf are not detected; they propagate.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,   /* NULL pointer, size < 1, bad flag, scale not finite or <= 0 */
+    FA_ERR_UNSUPPORTED = 2,   /* head dim not 64/128, sizes beyond the limits, device not sm_100 */
+    FA_ERR_MISALIGNED = 3,    /* q/k/v/o not 16-byte aligned, lse not 4-byte aligned */
+    FA_ERR_LAUNCH = 4,        /* the CUDA runtime refused the launch (see fa_last_cuda_error) */
+    FA_ERR_TIMEOUT = 5,       /* a kernel-side wait gave up (reported by fa_get_device_status) */
+    FA_ERR_NO_DEVICE = 6      /* no usable CUDA device is current */
+} fa_status;
+
+/*
+ * fa_fwd -- exact attention forward, O and the per-row log-sum-exp.
+ *
+ *  q, k, v : const bf16 [B][H][N][d], contiguous, d innermost (the
+ *            (batch, heads, seq_len, head_dim) layout of the "Try It
+ *            Yourself" script of the FlashAttention explainer page).
+ *  o       : bf16 [B][H][N][d], contiguous; O = softmax(S) V rounded to bf16
+ *            (round-to-nearest-even).
+ *  lse     : float [B][H][N]; lse[b][h][i] = ln sum_j exp(S_ij) over the
+ *            allowed keys, natural-log units, scale included.  It is the
+ *            O(N) per-row statistic ("m and l") that the page keeps for a
+ *            backward pass that recomputes P ("Sizing a tile, and why the
+ *            backward pass recomputes instead of storing").
+ *  B, H, N : batch, heads, sequence length; each >= 1.  N need not be a
+ *            multiple of the tile size.  B*H <= 2^31-1, N <= 2^30.
+ *  d       : head dimension, 64 or 128 (else FA_ERR_UNSUPPORTED).
+ *  causal  : 0 = no mask, 1 = key j allowed for query i iff j <= i.
+ *  scale   : multiplier of Q K^T, finite and > 0 (usually 1/sqrt(d)).
+ *  stream  : cudaStream_t as void*.
+ *
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_MISALIGNED are
+ * returned before any device work; FA_ERR_NO_DEVICE if no device is
+ * current; FA_ERR_LAUNCH if the launch fails.  The buffers q/k/v/o/lse must
+ * not overlap o or lse.  Uses no device memory besides its arguments.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * fa_fwd_debug -- fa_fwd with the kernel watchdog exposed, for tests.
+ *
+ *  watchdog_ms : every wait inside the kernel gives up after this many
+ *                milliseconds (0 = the default of 4000 ms); the CTA then
+ *                records FA_ERR_TIMEOUT in the device status word, stops
+ *                issuing work, waits (bounded) for its own copies and
+ *                tensor-core operations in flight, frees its tensor memory
+ *                and exits.  The context stays usable.
+ *  inject      : 0 = normal run.  1 = the producer of the first CTA never
+ *                issues its first K-tile copy, so the consumer's wait can
+ *                only end by the watchdog (host-chosen fault injection; no
+ *                fault, trap or bad address is involved).
+ * Other arguments and errors as fa_fwd.  O and LSE are undefined when the
+ * watchdog fires.
+ */
+fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int H, int N, int d, int causal, float scale, void* stream,
+                       unsigned watchdog_ms, int inject);
+
+/*
+ * fa_get_device_status -- read and clear the device status word of the
+ * current device.  Synchronises `stream` first.  Returns FA_OK or
+ * FA_ERR_TIMEOUT (a kernel watchdog fired since the last read); *detail, if
+ * not NULL, receives the raw word (role and unit of the first timeout).
+ * Returns FA_ERR_NO_DEVICE / FA_ERR_LAUNCH if the CUDA calls fail.
+ */
+fa_status fa_get_device_status(void* stream, unsigned* detail);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(int status);
+
+/* cudaError_t value behind the last FA_ERR_LAUNCH / FA_ERR_NO_DEVICE in this thread. */
+int fa_last_cuda_error(void);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

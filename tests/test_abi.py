@@ -1,0 +1,85 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol that
+include/fa.h declares, and rejects bad arguments before touching a device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_122_b200 as fa
+from exact_attention_122_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    fa_build.build()
+    return fa.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_exports():
+    assert declared_functions() == sorted(fa.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fa.library_path())
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version():
+    for code, name in [(0, "FA_OK"), (1, "FA_ERR_INVALID_ARG"), (2, "FA_ERR_UNSUPPORTED"),
+                       (3, "FA_ERR_MISALIGNED"), (4, "FA_ERR_LAUNCH"), (5, "FA_ERR_TIMEOUT"),
+                       (6, "FA_ERR_NO_DEVICE")]:
+        assert fa.status_string(code) == name
+    assert fa.status_string(99) == "FA_ERR_UNKNOWN"
+    assert fa.version() >= 100
+
+
+# Fake, never-dereferenced addresses: validation happens before any device
+# work, so these calls are safe without a GPU.
+P = 1 << 20
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((0, P, P, P, P, 1, 1, 8, 64, 0, 1.0), fa.FA_ERR_INVALID_ARG),        # NULL q
+    ((P, P, P, P, 0, 1, 1, 8, 64, 0, 1.0), fa.FA_ERR_INVALID_ARG),        # NULL lse
+    ((P, P, P, P, P, 0, 1, 8, 64, 0, 1.0), fa.FA_ERR_INVALID_ARG),        # B = 0
+    ((P, P, P, P, P, 1, -2, 8, 64, 0, 1.0), fa.FA_ERR_INVALID_ARG),       # H < 0
+    ((P, P, P, P, P, 1, 1, 0, 64, 0, 1.0), fa.FA_ERR_INVALID_ARG),        # N = 0
+    ((P, P, P, P, P, 1, 1, 8, 64, 2, 1.0), fa.FA_ERR_INVALID_ARG),        # causal flag
+    ((P, P, P, P, P, 1, 1, 8, 64, 0, 0.0), fa.FA_ERR_INVALID_ARG),        # scale 0
+    ((P, P, P, P, P, 1, 1, 8, 64, 0, -1.0), fa.FA_ERR_INVALID_ARG),       # scale < 0
+    ((P, P, P, P, P, 1, 1, 8, 64, 0, float("nan")), fa.FA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, 1, 1, 8, 64, 0, float("inf")), fa.FA_ERR_INVALID_ARG),
+    ((P, P, P, P, P, 1, 1, 8, 96, 0, 1.0), fa.FA_ERR_UNSUPPORTED),        # d = 96
+    ((P, P, P, P, P, 1, 1, 8, 256, 0, 1.0), fa.FA_ERR_UNSUPPORTED),       # d = 256
+    ((P, P, P, P, P, 1, 1, (1 << 30) + 1, 64, 0, 1.0), fa.FA_ERR_UNSUPPORTED),
+    ((P, P, P, P, P, 1 << 16, 1 << 16, 8, 64, 0, 1.0), fa.FA_ERR_UNSUPPORTED),  # B*H > 2^31-1
+    ((P + 8, P, P, P, P, 1, 1, 8, 64, 0, 1.0), fa.FA_ERR_MISALIGNED),     # q not 16-B aligned
+    ((P, P, P + 2, P, P, 1, 1, 8, 128, 1, 1.0), fa.FA_ERR_MISALIGNED),    # v
+    ((P, P, P, P + 4, P, 1, 1, 8, 64, 0, 1.0), fa.FA_ERR_MISALIGNED),     # o
+    ((P, P, P, P, P + 2, 1, 1, 8, 64, 0, 1.0), fa.FA_ERR_MISALIGNED),     # lse not 4-B aligned
+])
+def test_argument_validation(args, expect):
+    assert fa.fa_fwd_raw(*args, 0) == expect
+
+
+def test_debug_entry_validates_inject():
+    assert fa.fa_fwd_debug_raw(P, P, P, P, P, 1, 1, 8, 64, 0, 1.0, 0, 100, 7) == fa.FA_ERR_INVALID_ARG
+
+
+def test_python_wrapper_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.fa_fwd(q, q, q)

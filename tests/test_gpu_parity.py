@@ -1,0 +1,263 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (fixed for this path): max |dO| <= 2e-2, RMS dO <= 2e-3,
+max |dLSE| <= 1e-3, on the same seeded bf16 inputs.  Small and medium
+workloads are compared element by element; the two long-context workloads are
+run at full size in the launch configuration bench.py times and compared on
+sampled rows the oracle computes one by one, plus properties that hold at any
+size (every output finite; causal row 0 returns v_0 exactly).
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL_MAX = 2e-2
+TOL_RMS = 2e-3
+TOL_LSE = 1e-3
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module")
+def fa():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    import exact_attention_122_b200 as m
+    from exact_attention_122_b200 import build
+    build.build()
+    return m
+
+
+def run(fa, q, k, v, causal, scale, stream=None):
+    qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
+    o, lse = fa.fa_fwd(qd, kd, vd, causal=causal, scale=scale, stream=stream)
+    torch.cuda.synchronize()
+    st, word = fa.device_status()
+    assert st == fa.FA_OK, f"device status {fa.status_string(st)} {word:#x}"
+    return o, lse
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check(o, lse, O_ref, L_ref, what=""):
+    O = f64(o)
+    L = lse.detach().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(O)) and np.all(np.isfinite(L)), what
+    d = np.abs(O - O_ref)
+    err_max, err_rms = float(d.max()), float(np.sqrt(np.mean(d * d)))
+    err_lse = float(np.abs(L - L_ref).max())
+    assert err_max <= TOL_MAX, f"{what} max|dO| {err_max}"
+    assert err_rms <= TOL_RMS, f"{what} rms dO {err_rms}"
+    assert err_lse <= TOL_LSE, f"{what} max|dLSE| {err_lse}"
+    return err_max, err_rms, err_lse
+
+
+# ---------------------------------------------------------------------------
+# The worked example of the "Flash attention optimization" chapter, embedded
+# in head dimension d: q = e0, k_j = s_j e0, v_j = v_j e0, scale 1.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d", [64, 128])
+def test_worked_example_embedded(fa, d):
+    g = json.load(open(os.path.join(GOLDEN, "online_softmax_worked_example.json")))
+    s, vals = g["scores"], g["values"]
+    n = len(s)
+    q = torch.zeros(1, 1, n, d); q[..., 0] = 1.0
+    k = torch.zeros(1, 1, n, d); k[0, 0, :, 0] = torch.tensor(s)
+    v = torch.zeros(1, 1, n, d); v[0, 0, :, 0] = torch.tensor(vals)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))      # 1,3,2,5,10..40 are exact in bf16
+    o, lse = run(fa, q, k, v, False, 1.0)
+    O = f64(o); L = lse.cpu().numpy()
+    # Every row sees the four scores: O[:, 0] is the page's 36.8806; bf16
+    # spacing at 32..64 is 0.25, so compare relative to 2^-8.
+    assert np.all(np.abs(O[0, 0, :, 0] - g["direct"]["O"]) <= g["direct"]["O"] * 2.0 ** -8)
+    assert np.all(O[0, 0, :, 1:] == 0.0)
+    assert np.all(np.abs(L[0, 0] - (5.0 + math.log(g["direct"]["sum"]))) <= TOL_LSE)
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=False, scale=1.0)
+    assert np.max(np.abs(O - O_ref) / np.maximum(np.abs(O_ref), 1.0)) <= 2.0 ** -8
+    assert np.max(np.abs(L - L_ref)) <= TOL_LSE
+    # causal: row i sees s_0..s_i
+    o, lse = run(fa, q, k, v, True, 1.0)
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=True, scale=1.0)
+    assert np.max(np.abs(f64(o) - O_ref) / np.maximum(np.abs(O_ref), 1.0)) <= 2.0 ** -8
+    assert np.max(np.abs(lse.cpu().numpy() - L_ref)) <= TOL_LSE
+
+
+# ---------------------------------------------------------------------------
+# The five workloads
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("index", [1, 2, 3])
+def test_workload_full(fa, index):
+    w = synth.workload(index)
+    q, k, v = synth.workload_qkv(w)
+    o, lse = run(fa, q, k, v, w.causal, w.scale)
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=w.causal, scale=w.scale)
+    check(o, lse, O_ref, L_ref, w.describe())
+
+
+def sample_rows(N, rng, extra=24):
+    fixed = [0, 1, 2, 127, 128, 129, 255, 256, 257, 383, 384, N // 2, N - 257, N - 256,
+             N - 129, N - 128, N - 127, N - 2, N - 1]
+    rows = set(r for r in fixed if 0 <= r < N)
+    rows.update(int(x) for x in rng.integers(0, N, size=extra))
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("index", [4, 5])
+def test_workload_full_size_sampled(fa, index):
+    w = synth.workload(index)
+    q, k, v = synth.workload_qkv(w)
+    o, lse = run(fa, q, k, v, w.causal, w.scale)
+    BH = w.B * w.H
+    o3 = o.view(BH, w.N, w.d)
+    lse2 = lse.view(BH, w.N)
+    # properties at any size
+    assert bool(torch.isfinite(o3).all()) and bool(torch.isfinite(lse2).all())
+    v3 = v.view(BH, w.N, w.d).to("cuda:0")
+    if w.causal:
+        assert torch.equal(o3[:, 0, :], v3[:, 0, :]), "causal row 0 must return v_0 exactly"
+    rng = np.random.default_rng(1234 + index)
+    q3, k3, vv3 = (t.view(BH, w.N, w.d) for t in (q, k, v))
+    heads = sorted(set([0, BH - 1, BH // 2] + [int(x) for x in rng.integers(0, BH, size=2)]))
+    diffs, lse_err = [], 0.0
+    for bh in heads:
+        rows = sample_rows(w.N, rng)
+        qb, kb, vb = (oracle.exact_attention._as_f64(t[bh]) for t in (q3, k3, vv3))
+        O_ref, L_ref = oracle.attention_rows_fp64(qb, kb, vb, rows, w.causal, w.scale)
+        O = f64(o3[bh, torch.from_numpy(rows).to("cuda:0")])
+        L = lse2[bh].cpu().numpy()[rows]
+        diffs.append(np.abs(O - O_ref))
+        lse_err = max(lse_err, float(np.abs(L - L_ref).max()))
+    d = np.concatenate(diffs)
+    assert d.max() <= TOL_MAX, d.max()
+    assert np.sqrt(np.mean(d * d)) <= TOL_RMS
+    assert lse_err <= TOL_LSE, lse_err
+
+
+# ---------------------------------------------------------------------------
+# Ragged and edge shapes
+# ---------------------------------------------------------------------------
+RAGGED_N = [1, 5, 64, 127, 128, 129, 200, 255, 256, 257, 300, 511, 513, 1000]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", RAGGED_N)
+def test_ragged(fa, N, d, causal):
+    q, k, v = synth.draw_qkv(2, 3, N, d, seed=7000 + N * 3 + d + int(causal))
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run(fa, q, k, v, causal, scale)
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=causal, scale=scale)
+    check(o, lse, O_ref, L_ref, f"N={N} d={d} causal={causal}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_peaked_scores_rescale_often(fa, d):
+    """Q, K ~ N(0, 3^2): scaled scores with std 9, the running max moves often."""
+    q, k, v = synth.draw_qkv(1, 2, 2048, d, seed=99, qk_std=3.0)
+    scale = 1.0 / math.sqrt(d)
+    for causal in (True, False):
+        o, lse = run(fa, q, k, v, causal, scale)
+        O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=causal, scale=scale)
+        check(o, lse, O_ref, L_ref, f"peaked d={d} causal={causal}")
+
+
+def test_many_short_units(fa):
+    """More units than SMs, each short: exercises the persistent unit loop."""
+    q, k, v = synth.draw_qkv(2, 150, 256, 64, seed=5)
+    for causal in (True, False):
+        o, lse = run(fa, q, k, v, causal, 0.125)
+        O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=causal, scale=0.125)
+        check(o, lse, O_ref, L_ref, f"many units causal={causal}")
+
+
+def test_nonstandard_scale(fa):
+    q, k, v = synth.draw_qkv(1, 2, 384, 128, seed=77)
+    for scale in (0.01, 0.3):
+        o, lse = run(fa, q, k, v, True, scale)
+        O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=True, scale=scale)
+        check(o, lse, O_ref, L_ref, f"scale={scale}")
+
+
+def test_deterministic(fa):
+    w = synth.workload(3)
+    q, k, v = synth.workload_qkv(w)
+    o1, l1 = run(fa, q, k, v, w.causal, w.scale)
+    o2, l2 = run(fa, q, k, v, w.causal, w.scale)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_writes_stay_in_bounds(fa):
+    """Outputs pre-filled with NaN and followed by canaries: every valid
+    element is written, nothing past the end is touched."""
+    B, H, N, d = 1, 3, 300, 128
+    q, k, v = synth.draw_qkv(B, H, N, d, seed=3)
+    qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
+    n_o, n_l, pad = B * H * N * d, B * H * N, 4096
+    o_buf = torch.full((n_o + pad,), float("nan"), dtype=torch.bfloat16, device="cuda:0")
+    l_buf = torch.full((n_l + pad,), float("nan"), dtype=torch.float32, device="cuda:0")
+    o_buf[n_o:] = 7.0
+    l_buf[n_l:] = 7.0
+    o = o_buf[:n_o].view(B, H, N, d)
+    lse = l_buf[:n_l].view(B, H, N)
+    fa.fa_fwd(qd, kd, vd, causal=True, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(o).all()) and bool(torch.isfinite(lse).all())
+    assert bool((o_buf[n_o:] == 7.0).all()) and bool((l_buf[n_l:] == 7.0).all())
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=True, scale=1 / math.sqrt(d))
+    check(o, lse, O_ref, L_ref, "canary case")
+
+
+def test_argument_errors_on_device(fa):
+    q = torch.zeros(1, 1, 64 * 128 + 8, dtype=torch.bfloat16, device="cuda:0")
+    base = q.data_ptr()
+    lse = torch.zeros(64, dtype=torch.float32, device="cuda:0")
+    s = torch.cuda.current_stream().cuda_stream
+    # misaligned by one element (2 bytes): refused before launch
+    assert fa.fa_fwd_raw(base + 2, base, base, base, lse.data_ptr(), 1, 1, 64, 128, 0, 0.1, s) \
+        == fa.FA_ERR_MISALIGNED
+    assert fa.fa_fwd_raw(base, base, base, base, lse.data_ptr(), 1, 1, 64, 80, 0, 0.1, s) \
+        == fa.FA_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert fa.device_status()[0] == fa.FA_OK
+
+
+def test_watchdog_reports_timeout_and_context_survives(fa):
+    """Host-chosen injection: one producer never issues a copy, so a consumer
+    wait can only end by the watchdog.  The kernel must report
+    FA_ERR_TIMEOUT through the status word, exit, and leave the context
+    usable for the next correct run."""
+    q, k, v = synth.draw_qkv(1, 2, 1024, 64, seed=11)
+    qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
+    o = torch.empty_like(qd)
+    lse = torch.empty(1, 2, 1024, dtype=torch.float32, device="cuda:0")
+    s = torch.cuda.current_stream().cuda_stream
+    st = fa.fa_fwd_debug_raw(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), 1, 2, 1024, 64, 1, 0.125, s, 100, 1)
+    assert st == fa.FA_OK
+    st, word = fa.device_status(s)
+    assert st == fa.FA_ERR_TIMEOUT, (st, hex(word))
+    assert (word >> 24) == fa.FA_ERR_TIMEOUT
+    # the next call runs normally
+    o2, l2 = run(fa, q, k, v, True, 0.125)
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=True, scale=0.125)
+    check(o2, l2, O_ref, L_ref, "after watchdog")
+
+
+def test_side_stream(fa):
+    q, k, v = synth.draw_qkv(2, 4, 640, 128, seed=21)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o, lse = run(fa, q, k, v, True, 1 / math.sqrt(128), stream=s)
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=True, scale=1 / math.sqrt(128))
+    check(o, lse, O_ref, L_ref, "side stream")
