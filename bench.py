@@ -1,0 +1,436 @@
+#!/usr/bin/env python3
+"""Benchmark: exact attention forward TFLOP/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one exact-attention forward (one fa_fwd launch) over one batch of
+the long-context causal workload (B=2, H=32, N=8192, d=128, bf16, seeded
+N(0,1) inputs), inputs resident in HBM.  FLOPs per step: 4*B*H*N^2*d / 2.
+Prints one JSON line (rank 0).
+
+For N > 1 (torchrun, one process per GPU) every rank runs its own batch of
+the same shape: the forward has no exchange step, so the ranks share nothing
+but the barrier and the max-over-ranks timing reduction (weak scaling).
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (the
+reference arm): each step is a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s and % of B200 dense BF16 peak (1 GPU)"
+UNIT = "TFLOP/s"
+WORKLOAD_INDEX = 4          # long-context causal: B=2, H=32, N=8192, d=128
+KERNEL_SOURCE = os.path.join(ROOT, "exact_attention_122_b200", "csrc", "fa_fwd_sm100.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAK_TFLOPS = 1590.0   # used only when the measured peaks file is absent
+
+
+# ---------------------------------------------------------------------------
+# Host-side helpers (also exercised by the CPU tests)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return world, rank, local
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch (independent problems, weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank float over the process group (identity if none)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sample_plan(w: synth.Workload, rows: int):
+    """Bounded oracle sample: the last ``rows`` query rows of head 0 (the
+    rows with the most allowed keys).  Returns (row indices, FLOPs)."""
+    rows = max(1, min(rows, w.N))
+    idx = list(range(w.N - rows, w.N))
+    if w.causal:
+        keys = sum(i + 1 for i in idx)
+    else:
+        keys = rows * w.N
+    return idx, 4.0 * keys * w.d
+
+
+def kernel_source_sha() -> str:
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0.0)), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_PEAK_TFLOPS, 0.0, "fallback"
+
+
+def load_traffic(workload_name: str):
+    """Per-launch DRAM bytes from the committed ncu summary, only while the
+    kernel source still matches the one that was profiled."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("kernel_source_sha256") != kernel_source_sha() or t.get("workload") != workload_name:
+        return None
+    return t.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown",
+        0x0000000000000010: "sync_boost",
+        0x0000000000000100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.ok = False
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            uuid = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                pass
+            self._h = None
+            if uuid:
+                try:
+                    self._h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+                except Exception:
+                    self._h = None
+            if self._h is None:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "source": "nvml unavailable" if not self.ok else "no samples"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = threadpool_info()
+        return max((i.get("num_threads", 0) for i in info), default=0)
+    except Exception:
+        return 0
+
+
+def time_oracle_sample(w: synth.Workload, q, k, v, target_s: float, max_rows: int | None = None):
+    """Time the fp64 oracle on the last rows of head 0 (bounded sample).
+
+    Grows the sample until it takes about ``target_s`` seconds.  Returns
+    (TFLOP/s, seconds, rows, description)."""
+    import numpy as np
+
+    import oracle
+
+    qb, kb, vb = (oracle.exact_attention._as_f64(t[0, 0]) for t in (q, k, v))
+    rows = 64
+    while True:
+        idx, flops = sample_plan(w, rows)
+        t0 = time.perf_counter()
+        oracle.attention_rows_fp64(qb, kb, vb, np.array(idx), w.causal, w.scale)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or rows >= w.N or (max_rows and rows >= max_rows):
+            break
+        grow = max(2.0, min(16.0, target_s / max(dt, 1e-3)))
+        rows = min(w.N, int(rows * grow))
+        if max_rows:
+            rows = min(rows, max_rows)
+    desc = (f"fp64 oracle (materialised S and P rows) on the last {len(idx)} query rows of head 0 "
+            f"of {w.describe()}, {flops / 1e9:.2f} GFLOP")
+    return flops / dt / 1e12, dt, len(idx), desc
+
+
+# ---------------------------------------------------------------------------
+# Reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if world > 1 and rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle
+
+    q, k, v = synth.workload_qkv(w)
+    qb, kb, vb = (oracle.exact_attention._as_f64(t[0, 0]) for t in (q, k, v))
+    steps_total = args.steps + args.warmup
+    per_step = max(0.05, min(2.0, 150.0 / max(1, steps_total)))
+    # calibrate the row count for ~per_step seconds
+    rows = 32
+    while True:
+        idx, flops = sample_plan(w, rows)
+        t0 = time.perf_counter()
+        oracle.attention_rows_fp64(qb, kb, vb, np.array(idx), w.causal, w.scale)
+        dt = time.perf_counter() - t0
+        if dt >= per_step * 0.7 or rows >= w.N:
+            break
+        rows = min(w.N, int(rows * max(1.5, min(8.0, per_step / max(dt, 1e-4)))))
+    idx, flops = sample_plan(w, rows)
+    idx = np.array(idx)
+    for _ in range(args.warmup):
+        oracle.attention_rows_fp64(qb, kb, vb, idx, w.causal, w.scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attention_rows_fp64(qb, kb, vb, idx, w.causal, w.scale)
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    cores = blas_threads() or os.cpu_count()
+    sample = (f"each step: fp64 oracle on the last {len(idx)} query rows of head 0 of "
+              f"{w.describe()} ({flops / 1e9:.2f} GFLOP)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: synth.Workload, n_gpus: int):
+    return {"workload": w.name, "B_per_gpu": w.B, "H": w.H, "N": w.N, "d": w.d,
+            "causal": w.causal, "scale": w.scale, "global_batch": w.B * n_gpus, "seq_len": w.N,
+            "parallelism": f"independent batches x{n_gpus}" if n_gpus > 1 else "single GPU",
+            "l2": f"inputs {3 * w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB > 126 MB L2; no flush"}
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_122_b200 as fa
+
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    q, k, v = synth.draw_qkv(w.B, w.H, w.N, w.d, rank_seed(w.seed, rank), w.qk_std)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    od = torch.empty_like(qd)
+    lsed = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        fa.fa_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=od, lse=lsed, stream=stream)
+
+    def sync_all():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    st, word = fa.device_status(stream.cuda_stream)
+    if st != fa.FA_OK:
+        raise SystemExit(f"kernel status {fa.status_string(st)} {word:#x}")
+
+    # --- device-timed region: K launches, per-launch events on the launch stream
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sync_all()
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            t_begin.record(stream)
+            for i in range(args.steps):
+                starts[i].record(stream)
+                step()
+                ends[i].record(stream)
+            t_end.record(stream)
+        sync_all()
+    total_ms = t_begin.elapsed_time(t_end)
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(total_ms, dev)
+    avg_launch_ms = max_over_ranks(sum(launch_ms) / len(launch_ms), dev)
+    st, word = fa.device_status(stream.cuda_stream)
+    if st != fa.FA_OK:
+        raise SystemExit(f"kernel status {fa.status_string(st)} {word:#x}")
+
+    flops_step = w.flops
+    ms_per_step = total_ms / args.steps
+    value = world * flops_step * args.steps / (total_ms / 1e3) / 1e12
+
+    # --- end to end through the public API: pinned host -> device, forward,
+    # device -> host of O and LSE, every step.
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        fa.fa_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=od, lse=lsed, stream=stream)
+        oh.copy_(od, non_blocking=True)
+        lh.copy_(lsed, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step()
+    sync_all()
+    e_begin = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e_begin.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e_end.record(stream)
+    sync_all()
+    e2e_ms = max_over_ranks(e_begin.elapsed_time(e_end), dev)
+    e2e_value = world * flops_step * e2e_steps / (e2e_ms / 1e3) / 1e12
+
+    peak, peak_sustained, peak_src = load_peaks()
+    achieved = flops_step / (avg_launch_ms / 1e3) / 1e12
+    traffic = load_traffic(w.name)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, world),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "frac_of_sustained": (achieved / peak_sustained) if peak_sustained else None,
+                     "kernel": "fa_fwd_kernel<128,4>", "avg_launch_ms": avg_launch_ms},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, secs, rows, desc = time_oracle_sample(w, q, k, v, target_s=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": blas_threads() or os.cpu_count(),
+                                "kind": "oracle", "sample": desc, "seconds": secs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=WORKLOAD_INDEX,
+                    help="workload index (1..5); the default is the headline workload")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target length of the oracle CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.steps < 1:
+        raise SystemExit("--steps must be >= 1")
+    w = synth.workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

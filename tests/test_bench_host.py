@@ -1,0 +1,105 @@
+"""Host-side logic of bench.py, on the CPU: the FLOP/byte bookkeeping, the
+oracle sample plan, the traffic lookup, and the multi-rank path (weak
+scaling: each rank its own batch; the only collectives are the barrier and the
+max-over-ranks timing reduction), run as two gloo ranks."""
+
+import json
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import synth
+
+
+def test_workload_bookkeeping():
+    w = synth.workload(4)
+    assert (w.B, w.H, w.N, w.d, w.causal) == (2, 32, 8192, 128, True)
+    assert w.flops == 4 * 2 * 32 * 8192 ** 2 * 128 / 2
+    assert w.algorithmic_bytes == 4 * 2 * 32 * 8192 * 128 * 2 + 2 * 32 * 8192 * 4
+    w1 = synth.workload(1)
+    assert w1.flops == 4 * 256 * 256 * 64 and not w1.causal
+    assert abs(synth.workload(5).scale - 1 / 128 ** 0.5) < 1e-15
+
+
+def test_sample_plan_counts_allowed_keys():
+    w = synth.workload(4)
+    idx, flops = bench.sample_plan(w, 3)
+    assert idx == [8189, 8190, 8191]
+    assert flops == 4.0 * (8190 + 8191 + 8192) * 128
+    w2 = synth.workload(2)
+    idx, flops = bench.sample_plan(w2, 10)
+    assert flops == 4.0 * 10 * 512 * 64
+
+
+def test_inputs_are_seeded_and_rank_distinct():
+    a = synth.draw_qkv(1, 2, 16, 64, seed=bench.rank_seed(1224, 0))
+    b = synth.draw_qkv(1, 2, 16, 64, seed=bench.rank_seed(1224, 0))
+    c = synth.draw_qkv(1, 2, 16, 64, seed=bench.rank_seed(1224, 1))
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    assert not torch.equal(a[0], c[0])
+    assert a[0].dtype == torch.bfloat16 and a[0].is_contiguous()
+
+
+def test_traffic_is_null_unless_kernel_matches(tmp_path, monkeypatch):
+    f = tmp_path / "t.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.load_traffic("long_context_causal") is None
+    f.write_text(json.dumps({"kernel_source_sha256": "0" * 64, "workload": "long_context_causal",
+                             "bytes_per_launch": 123}))
+    assert bench.load_traffic("long_context_causal") is None
+    f.write_text(json.dumps({"kernel_source_sha256": bench.kernel_source_sha(),
+                             "workload": "long_context_causal", "bytes_per_launch": 123}))
+    assert bench.load_traffic("long_context_causal") == 123
+    assert bench.load_traffic("other") is None
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w, r, lr = bench.dist_env()
+        per_rank_ms = [3.5, 7.25][rank]
+        m = bench.max_over_ranks(per_rank_ms)
+        seed = bench.rank_seed(1224, r)
+        dist.barrier()
+        out.put((rank, w, r, lr, m, seed))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_timing_reduction_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [2, 2]
+    assert [r[2] for r in res] == [0, 1]
+    assert all(r[4] == 7.25 for r in res)          # max over ranks, seen by every rank
+    assert res[0][5] != res[1][5]                   # independent batches per rank
+
+
+def test_single_process_max_is_identity():
+    assert bench.max_over_ranks(4.0) == 4.0
+
+
+def test_cli_rejects_short_warmup():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])
