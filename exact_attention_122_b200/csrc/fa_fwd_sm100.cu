@@ -70,6 +70,21 @@ constexpr int REGS_OTHER = 80;
 static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER <= NUM_THREADS * REGS_LAUNCH,
               "register split exceeds the launch allocation");
 constexpr int SW_COLS = 64;        // bf16 elements per 128-byte swizzled row
+// Lazy rescale: the running max that l and O refer to is only moved when a
+// row's new maximum exceeds it by more than RESCALE_LOG2 (log2 units), so P
+// stays below 2^RESCALE_LOG2 and O is rescaled rarely.  l and O share the
+// stale reference, so O = acc / l and LSE = (m + log2 l) ln 2 stay exact.
+constexpr float RESCALE_LOG2 = 8.0f;
+// Columns of every 32-column chunk of an unmasked score row whose
+// exponential is computed by exp2_poly instead of MUFU ex2.
+// Measured on B200: every nonzero setting was slower on the long causal
+// workloads (the softmax is not MUFU-bound once the rescale is lazy), so the
+// default is 0; the polynomial path stays for tuning other shapes.
+#ifndef FA_POLY_COLS
+#define FA_POLY_COLS 0
+#endif
+constexpr int POLY_COLS = FA_POLY_COLS;
+static_assert(POLY_COLS >= 0 && POLY_COLS <= 32 && POLY_COLS % 2 == 0, "poly columns");
 
 enum : uint32_t {
     ROLE_SOFTMAX = 1u, ROLE_MMA = 2u, ROLE_PRODUCER = 3u, ROLE_DRAIN = 4u
@@ -245,6 +260,41 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
+// 128 consecutive 32-bit TMEM columns of this thread's lane (one full score
+// row), waited on inside the same asm statement.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+        "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, "
+        "%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
+        "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, "
+        "%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, "
+        "%112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127 "
+        "}, [%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]),
+          "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]),
+          "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]),
+          "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]),
+          "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]),
+          "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]),
+          "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]),
+          "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]),
+          "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+        : "r"(taddr)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -293,6 +343,30 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Software 2^x on the FMA pipe, used for part of each score row so the
+// MUFU unit (ex2) is not the only source of exponentials.  Method:
+// Cody-Waite range reduction x = n + f with n = rint(x) (the 1.5 * 2^23
+// rounding constant), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
+// exchange; csrc/gen_exp2_poly.py reproduces them, max relative error
+// 7.5e-5, below the 2^-9 rounding of the bf16 P it feeds); 2^n is added to
+// the exponent field.  Valid for x in [-126, 64]; inputs below -126 are
+// clamped (results below 2^-125 are meaningless there, so the kernel only
+// uses it on tiles without masked scores).
+constexpr float EXP2_C0 = 9.999280572e-01f;
+constexpr float EXP2_C1 = 6.932609677e-01f;
+constexpr float EXP2_C2 = 2.426111251e-01f;
+constexpr float EXP2_C3 = 5.517166853e-02f;
+
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -126.0f);
+    const float t = x + 12582912.0f;            // 1.5 * 2^23: t's low bits hold rint(x)
+    const float n = t - 12582912.0f;
+    const float f = x - n;
+    const float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, EXP2_C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
     return *reinterpret_cast<uint32_t*>(&h);
@@ -320,20 +394,31 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
 }
 
 // ---------------------------------------------------------------------------
-// Work decomposition: units of 256 query rows of one (batch, head).  Unit u
-// is (level, bh) with level = u / BH; for causal masking the level counts
-// down from the last (longest) row block so the longest units go first.
+// Work decomposition: units of 256 query rows of one (batch, head).
+// Units are ordered in groups of `hg` heads (sized on the host so a group's
+// K and V stay resident in L2 while the CTAs working on it stream them);
+// inside a group the order is by row block, the longest causal rows first.
+// CTA b takes sequence indices in boustrophedon order (b, 2S-1-b, 2S+b, ...)
+// so long and short units pair up across CTAs.
 // ---------------------------------------------------------------------------
 struct Unit {
     int bh, r0, nb0, nb1;  // first row, K/V tile counts of sub-tiles 0 and 1
 };
 
-__device__ __forceinline__ Unit decode_unit(int u, int BH, int N, int causal) {
+__device__ __forceinline__ int unit_index(int k, int cta, int ctas) {
+    return k * ctas + ((k & 1) ? (ctas - 1 - cta) : cta);
+}
+
+__device__ __forceinline__ Unit decode_unit(int i, int BH, int N, int causal, int hg) {
     const int nq2 = (N + UNIT_ROWS - 1) / UNIT_ROWS;
     const int nkb = (N + BN - 1) / BN;
-    const int level = u / BH;
+    const int per_group = hg * nq2;
+    const int g = i / per_group;
+    const int r = i - g * per_group;
+    const int gh = min(hg, BH - g * hg);       // heads in this group
+    const int level = r / gh;
     Unit w;
-    w.bh = u - level * BH;
+    w.bh = g * hg + (r - level * gh);
     const int qb2 = causal ? (nq2 - 1 - level) : level;
     w.r0 = qb2 * UNIT_ROWS;
     if (causal) {
@@ -346,6 +431,35 @@ __device__ __forceinline__ Unit decode_unit(int u, int BH, int N, int causal) {
     return w;
 }
 
+// P = 2^(s * scale_log2 - m) for one score row held in registers, written
+// to TMEM as bf16 pairs over the row's first 64 columns; the row sum goes to
+// four partial accumulators.  The first NPOLY columns of every 32-column
+// chunk use exp2_poly, the rest MUFU ex2.
+template <int NPOLY>
+__device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_log2, float neg_m,
+                                             float (&rs)[4], uint32_t tS) {
+#pragma unroll
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float x0 = fmaf(s[c * 32 + 2 * i], scale_log2, neg_m);
+            const float x1 = fmaf(s[c * 32 + 2 * i + 1], scale_log2, neg_m);
+            float p0, p1;
+            if (2 * i < NPOLY) {
+                p0 = exp2_poly(x0);
+                p1 = exp2_poly(x1);
+            } else {
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+            }
+            rs[i & 3] += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + c * 16, pk);              // P (bf16) over S columns [0, 64)
+    }
+}
+
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
@@ -354,7 +468,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ Og,
                   float* __restrict__ LSEg, int BH, int N, int causal, float scale_log2,
-                  unsigned long long watchdog_ns, int inject) {
+                  int hg, unsigned long long watchdog_ns, int inject) {
     using L = Layout<D, NS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -418,8 +532,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int s = 0; s < NS; ++s) stage_fill[s] = 0;
             bool ok = true;
             bool skipped = false;
-            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++units) {
-                const Unit w = decode_unit(u, BH, N, causal);
+            for (int kq = 0, u; (u = unit_index(kq, blockIdx.x, gridDim.x)) < num_units && ok;
+                 ++kq, ++units) {
+                const Unit w = decode_unit(u, BH, N, causal, hg);
                 if (!wait_phase(bar(L::B_Q_EMPTY), (units & 1u) ^ 1u, wd, ROLE_PRODUCER, u)) {
                     ok = false;
                     break;
@@ -507,8 +622,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                            ID_PV, (first && kk == 0) ? 0u : 1u);
                 }
             };
-            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++units) {
-                const Unit w = decode_unit(u, BH, N, causal);
+            for (int kq = 0, u; (u = unit_index(kq, blockIdx.x, gridDim.x)) < num_units && ok;
+                 ++kq, ++units) {
+                const Unit w = decode_unit(u, BH, N, causal, hg);
                 if (!wait_phase(bar(L::B_Q_FULL), units & 1u, wd, ROLE_MMA, u)) { ok = false; break; }
                 uint32_t sK = cons % NS;
                 if (!wait_phase(bar(L::B_KV_FULL + sK), (cons / NS) & 1u, wd, ROLE_MMA, u)) {
@@ -612,8 +728,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t tO = tmem + lane_base + (t == 0 ? L::TM_O0 : L::TM_O1);
         uint32_t scnt = 0, ocnt = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-            const Unit w = decode_unit(u, BH, N, causal);
+        for (int kq = 0, u; (u = unit_index(kq, blockIdx.x, gridDim.x)) < num_units && ok; ++kq) {
+            const Unit w = decode_unit(u, BH, N, causal, hg);
             const int a = w.r0 + t * BM;             // first row of this sub-tile
             const int row = a + wr;
             const int nb = t == 0 ? w.nb0 : w.nb1;
@@ -625,12 +741,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
                 float s[BN];
+                {
+                    uint32_t r[BN];
+                    tmem_ld128(tS, r);
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + c * 32, r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+                    for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
                 }
                 // Mask: keys beyond N on the last tile; keys above the
                 // diagonal on a sub-tile's diagonal tile.
@@ -645,40 +760,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         s[c] = bad ? -INFINITY : s[c];
                     }
                 }
-                float mx = s[0];
+                // Row max: eight independent chains, then a tree.
+                float mx8[8];
 #pragma unroll
-                for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-                const float m_new = fmaxf(m, mx * scale_log2);
-                const float alpha = ex2(m - m_new);          // 0 on the first tile (m = -inf)
-                if (j > 0 && __any_sync(0xffffffffu, m_new > m)) {
-                    // Rescale this warp's rows of O (the PV of tile j-1 is
-                    // complete: its commit preceded the S_t commit above).
+                for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(tO + c * 32, r);
+                for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+                const float m_blk =
+                    fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+                // Lazy rescale (first tile: m = -inf, so every lane moves).
+                if (__any_sync(0xffffffffu, m_blk > m + RESCALE_LOG2)) {
+                    const float m_new = fmaxf(m, m_blk);
+                    const float alpha = ex2(m - m_new);      // 0 on the first tile
+                    if (j > 0) {
+                        // The PV of tile j-1 is complete: its commit
+                        // preceded the S_t commit waited on above.
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                        tmem_st32(tO + c * 32, r);
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t r[32];
+                            tmem_ld32(tO + c * 32, r);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                            tmem_st32(tO + c * 32, r);
+                        }
                     }
+                    l *= alpha;
+                    m = m_new;
                 }
-                l *= alpha;
-                m = m_new;
                 const float neg_m = -m;
-                float rowsum = 0.f;
-#pragma unroll
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float p0 = ex2(fmaf(s[c * 32 + 2 * i], scale_log2, neg_m));
-                        const float p1 = ex2(fmaf(s[c * 32 + 2 * i + 1], scale_log2, neg_m));
-                        rowsum += p0 + p1;
-                        pk[i] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(tS + c * 16, pk);              // P (bf16) over S columns [0, 64)
-                }
-                l += rowsum;
+                float rs[4] = {0.f, 0.f, 0.f, 0.f};
+                // Tiles without masked scores may use the FMA-pipe 2^x for
+                // part of the row; the choice is warp-uniform, made once.
+                if (POLY_COLS > 0 && !(tail || diag))
+                    exp_row_to_p<POLY_COLS>(s, scale_log2, neg_m, rs, tS);
+                else
+                    exp_row_to_p<0>(s, scale_log2, neg_m, rs, tS);
+                l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(L::B_P_FULL + t));
@@ -692,20 +811,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float inv_l = 1.f / l;
             const bool store = row < N;
             __nv_bfloat16* orow = Og + (size_t(w.bh) * N + (store ? row : 0)) * D;
+            uint32_t ro[D];
+            if constexpr (D == 128) {
+                tmem_ld128(tO, ro);
+            } else {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tO + c * 32, r);
-                uint32_t pk[16];
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tO + c * 32, r);
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
-                                        __uint_as_float(r[2 * i + 1]) * inv_l);
-                if (store) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                    for (int i = 0; i < 32; ++i) ro[c * 32 + i] = r[i];
+                }
+            }
+            if (store) {
+                uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                for (int v4 = 0; v4 < D / 8; ++v4) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(ro[8 * v4 + 2 * i]) * inv_l,
+                                            __uint_as_float(ro[8 * v4 + 2 * i + 1]) * inv_l);
+                    dst[v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
             if (store) LSEg[size_t(w.bh) * N + row] = (m + log2f(l)) * 0.69314718055994530942f;
@@ -800,11 +927,22 @@ fa_status launch(const void* q, const void* k, const void* v, void* o, float* ls
         return FA_ERR_UNSUPPORTED;
     const long long nq2 = (N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
     const long long units = nq2 * BH;
+    // Heads per scheduling group.  When all of K and V fit in 32 MiB of L2
+    // there is nothing to group and the whole problem is one group (best
+    // balance); otherwise groups of two heads keep the K/V that concurrently
+    // running CTAs stream resident in L2 (measured best on the 8K and 32K
+    // causal workloads).
+    const long long kv_head_bytes = 2LL * N * D * 2;
+    long long hg = (BH * kv_head_bytes <= (32LL << 20)) ? BH : 2;
+#ifdef FA_HEAD_GROUP
+    hg = FA_HEAD_GROUP;
+#endif
+    hg = hg < 1 ? 1 : (hg > BH ? BH : hg);
     const int grid = int(units < g_dev[dev].sm_count ? units : g_dev[dev].sm_count);
     const float scale_log2 = scale * 1.4426950408889634f;
     kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o),
                                                      lse, int(BH), N, causal, scale_log2,
-                                                     watchdog_ns, inject);
+                                                     int(hg), watchdog_ns, inject);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         t_last_cuda_error = int(e);
