@@ -221,15 +221,16 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
         : "memory");
 }
-// D(tmem) (+)= A(smem desc) * B(smem desc)
+// D(tmem) (+)= A(smem desc) * B(smem desc).  No "memory" clobber: the
+// operands are ordered by the (volatile, clobbering) mbarrier waits and
+// fences around the issue loops, and volatile asm keeps issue order.
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 // D(tmem) (+)= A(tmem) * B(smem desc)
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -238,8 +239,7 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // 32 consecutive 32-bit TMEM columns of this thread's lane, waited on inside
@@ -372,6 +372,28 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes of
+// work, each rounded exactly like its scalar counterpart).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+
 // ---- UMMA descriptors ----
 // Shared-memory matrix descriptor, 128-byte swizzle (the layout TMA writes
 // with CU_TENSOR_MAP_SWIZZLE_128B): start address, leading and stride byte
@@ -431,20 +453,53 @@ __device__ __forceinline__ Unit decode_unit(int i, int BH, int N, int causal, in
     return w;
 }
 
+// S = Q K^T for one sub-tile: M=128 query rows, N=128 keys, K=d in steps
+// of 16.  Both operands K-major with 128-byte swizzle: a step is 32 bytes
+// inside a swizzled row, and 64-column slabs are HALF_BYTES apart.  Adding
+// (offset >> 4) to a descriptor moves its start address by offset.
+// The start-address field (bits 0-13) never carries into the rest of the
+// descriptor for addresses below 256 KiB, so only the low word changes.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t off16) {
+    return (desc & 0xFFFFFFFF00000000ull) | uint64_t(uint32_t(desc) + off16);
+}
+
+template <int D, int HALF_BYTES>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc,
+                                         uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = uint32_t(((kk / 4) * HALF_BYTES + (kk % 4) * 32) >> 4);
+        mma_ss(d_tmem, desc_add(q_desc, off), desc_add(k_desc, off), idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+// O += P V for one sub-tile: A = P from TMEM (16 keys = 8 columns of bf16
+// pairs per step), B = V MN-major (16 key rows of 128 bytes per step).
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc,
+                                         uint32_t idesc, bool first) {
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk) {
+        const uint32_t off = uint32_t((kk * 16 * 128) >> 4);
+        mma_ts(o_tmem, p_tmem + kk * 8, desc_add(v_desc, off), idesc, (first && kk == 0) ? 0u : 1u);
+    }
+}
+
 // P = 2^(s * scale_log2 - m) for one score row held in registers, written
 // to TMEM as bf16 pairs over the row's first 64 columns; the row sum goes to
-// four partial accumulators.  The first NPOLY columns of every 32-column
-// chunk use exp2_poly, the rest MUFU ex2.
+// four packed partial accumulators.  The first NPOLY columns of every
+// 32-column chunk use exp2_poly, the rest MUFU ex2.
 template <int NPOLY>
 __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_log2, float neg_m,
-                                             float (&rs)[4], uint32_t tS) {
+                                             uint64_t (&acc)[4], uint32_t tS) {
+    const uint64_t c2 = f2_pack(scale_log2, scale_log2);
+    const uint64_t m2 = f2_pack(neg_m, neg_m);
 #pragma unroll
     for (int c = 0; c < BN / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            const float x0 = fmaf(s[c * 32 + 2 * i], scale_log2, neg_m);
-            const float x1 = fmaf(s[c * 32 + 2 * i + 1], scale_log2, neg_m);
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), c2, m2), x0, x1);
             float p0, p1;
             if (2 * i < NPOLY) {
                 p0 = exp2_poly(x0);
@@ -453,7 +508,7 @@ __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_l
                 p0 = ex2(x0);
                 p1 = ex2(x1);
             }
-            rs[i & 3] += p0 + p1;
+            acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
             pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + c * 16, pk);              // P (bf16) over S columns [0, 64)
@@ -479,6 +534,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t sBar = sbase + L::OFF_BAR;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    // Always 0: the abort flag of the drain waits, which must not be cut
+    // short by the CTA's own abort.
+    volatile int* zero_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);
     auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
 
     const int warp = threadIdx.x >> 5;
@@ -502,6 +560,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = 0;
+        *zero_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -528,10 +587,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // ------------------------------------------------------------------
         if (lane == 0) {
             uint32_t fills = 0, units = 0, q_issued = 0;
-            uint32_t stage_fill[NS];        // last fill index issued into each stage, +1
-            for (int s = 0; s < NS; ++s) stage_fill[s] = 0;
             bool ok = true;
-            bool skipped = false;
+            bool skipped = false;           // fault injection: fill 0 was never issued
             for (int kq = 0, u; (u = unit_index(kq, blockIdx.x, gridDim.x)) < num_units && ok;
                  ++kq, ++units) {
                 const Unit w = decode_unit(u, BH, N, causal, hg);
@@ -562,21 +619,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             for (int h = 0; h < D / SW_COLS; ++h)
                                 tma_load_3d(sKV + s * L::KV_BYTES + h * L::HALF_BYTES, map,
                                             h * SW_COLS, j * BN, w.bh, bar(L::B_KV_FULL + s));
-                            stage_fill[s] = fills + 1;
                         }
                         ++fills;
                     }
                 }
             }
             if (!ok) {
-                // Drain: wait (bounded) for every copy this thread issued.
-                Watchdog dwd{abort_flag, wd.limit_ns};
-                volatile int never = 0;
-                dwd.abort_flag = &never;
-                for (int s = 0; s < NS; ++s)
-                    if (stage_fill[s] != 0)
-                        wait_phase(bar(L::B_KV_FULL + s), ((stage_fill[s] - 1) / NS) & 1u, dwd,
-                                   ROLE_DRAIN, 0);
+                // Drain: wait (bounded) for every copy this thread issued:
+                // the last fill of each stage, f = fills-1-((fills-1-s) mod NS).
+                const Watchdog dwd{zero_flag, wd.limit_ns};
+                for (uint32_t s = 0; s < NS; ++s) {
+                    if (fills <= s) continue;
+                    const uint32_t f = fills - 1 - ((fills - 1 - s) % NS);
+                    if (skipped && f == 0) continue;
+                    wait_phase(bar(L::B_KV_FULL + s), (f / NS) & 1u, dwd, ROLE_DRAIN, 0);
+                }
                 if (q_issued > 0)
                     wait_phase(bar(L::B_Q_FULL), (q_issued - 1) & 1u, dwd, ROLE_DRAIN, 0);
             }
@@ -596,32 +653,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t cons = 0, units = 0, pcnt0 = 0, pcnt1 = 0;
             bool ok = true;
             bool issued = false;
-            auto issue_s = [&](int t, uint32_t kstage) {
-                const uint32_t dS = tmem + (t ? L::TM_S1 : L::TM_S0);
-                const uint32_t qa = sQ + t * L::Q_BYTES;
-                const uint32_t ka = sKV + kstage * L::KV_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    // K-major operands: 16 bf16 of d per MMA; 32 bytes inside a
-                    // 128-byte swizzled row, 64-column slabs 16 KiB apart.
-                    const uint32_t off = (kk / 4) * L::HALF_BYTES + (kk % 4) * 32;
-                    mma_ss(dS, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                           ID_S, kk > 0 ? 1u : 0u);
-                }
-            };
-            auto issue_pv = [&](int t, uint32_t vstage, bool first) {
-                const uint32_t dO = tmem + (t ? L::TM_O1 : L::TM_O0);
-                const uint32_t aP = tmem + (t ? L::TM_S1 : L::TM_S0);
-                const uint32_t va = sKV + vstage * L::KV_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    // A = P from TMEM (16 keys = 8 columns of bf16 pairs); B = V,
-                    // MN-major: 16 key rows of 128 bytes per step, d slabs 16 KiB
-                    // apart (leading byte offset), 8-row groups 1 KiB apart.
-                    mma_ts(dO, aP + kk * 8, sdesc_sw128(va + kk * 16 * 128, L::HALF_BYTES, 1024),
-                           ID_PV, (first && kk == 0) ? 0u : 1u);
-                }
-            };
+            // Descriptors, built once: Q sub-tiles and ring stages (K-major
+            // view for K, MN-major view for V: leading byte offset = the
+            // 16 KiB between d slabs, stride byte offset = 8 rows x 128 B).
+            const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
+            const uint64_t dq1 = sdesc_sw128(sQ + L::Q_BYTES, 16, 1024);
+            const uint64_t dk0 = sdesc_sw128(sKV, 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(sKV, L::HALF_BYTES, 1024);
+            const uint32_t stage_step = uint32_t(L::KV_BYTES >> 4);
+            const uint32_t tS0 = tmem + L::TM_S0, tS1 = tmem + L::TM_S1;
+            const uint32_t tO0 = tmem + L::TM_O0, tO1 = tmem + L::TM_O1;
             for (int kq = 0, u; (u = unit_index(kq, blockIdx.x, gridDim.x)) < num_units && ok;
                  ++kq, ++units) {
                 const Unit w = decode_unit(u, BH, N, causal, hg);
@@ -632,9 +673,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 }
                 ++cons;
-                issue_s(0, sK);
+                issue_qk<D, L::HALF_BYTES>(tS0, dq0, desc_add(dk0, sK * stage_step), ID_S);
                 tc_commit(bar(L::B_S_FULL + 0));
-                issue_s(1, sK);
+                issue_qk<D, L::HALF_BYTES>(tS1, dq1, desc_add(dk0, sK * stage_step), ID_S);
                 tc_commit(bar(L::B_S_FULL + 1));
                 tc_commit(bar(L::B_KV_EMPTY + sK));
                 issued = true;
@@ -667,9 +708,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         }
                         ++pcnt0;
                         tc_fence_after();
-                        issue_pv(0, sV, j == 0);
+                        issue_pv(tO0, tS0, desc_add(dv0, sV * stage_step), ID_PV, j == 0);
                         if (j + 1 < w.nb0) {
-                            issue_s(0, sK);
+                            issue_qk<D, L::HALF_BYTES>(tS0, dq0, desc_add(dk0, sK * stage_step), ID_S);
                             tc_commit(bar(L::B_S_FULL + 0));
                         }
                         if (j == w.nb0 - 1) tc_commit(bar(L::B_O_FULL + 0));
@@ -684,9 +725,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     ++pcnt1;
                     tc_fence_after();
-                    issue_pv(1, sV, j == 0);
+                    issue_pv(tO1, tS1, desc_add(dv0, sV * stage_step), ID_PV, j == 0);
                     if (next) {
-                        issue_s(1, sK);
+                        issue_qk<D, L::HALF_BYTES>(tS1, dq1, desc_add(dk0, sK * stage_step), ID_S);
                         tc_commit(bar(L::B_S_FULL + 1));
                     }
                     tc_commit(bar(L::B_KV_EMPTY + sV));
@@ -699,9 +740,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // Every MMA this thread issued must finish before TMEM is
                 // freed; on the normal path the softmax warps have already
                 // waited for the last O commit, so this returns at once.
-                Watchdog dwd{abort_flag, wd.limit_ns};
-                volatile int never = 0;
-                dwd.abort_flag = &never;
+                const Watchdog dwd{zero_flag, wd.limit_ns};
                 tc_commit(bar(L::B_DRAIN));
                 wait_phase(bar(L::B_DRAIN), 0, dwd, ROLE_DRAIN, 0);
             }
@@ -760,7 +799,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         s[c] = bad ? -INFINITY : s[c];
                     }
                 }
-                // Row max: eight independent chains, then a tree.
+                // Row max: eight independent chains, then a tree.  (The
+                // three-input max.f32 form measured inexact here: it broke the
+                // bit-exact causal row 0 of the parity tests.)
                 float mx8[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) mx8[i] = s[i];
@@ -790,14 +831,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     m = m_new;
                 }
                 const float neg_m = -m;
-                float rs[4] = {0.f, 0.f, 0.f, 0.f};
+                uint64_t acc[4] = {0, 0, 0, 0};              // four packed (0.f, 0.f)
                 // Tiles without masked scores may use the FMA-pipe 2^x for
                 // part of the row; the choice is warp-uniform, made once.
                 if (POLY_COLS > 0 && !(tail || diag))
-                    exp_row_to_p<POLY_COLS>(s, scale_log2, neg_m, rs, tS);
+                    exp_row_to_p<POLY_COLS>(s, scale_log2, neg_m, acc, tS);
                 else
-                    exp_row_to_p<0>(s, scale_log2, neg_m, rs, tS);
-                l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+                    exp_row_to_p<0>(s, scale_log2, neg_m, acc, tS);
+                {
+                    float a0, a1, a2, a3, a4, a5, a6, a7;
+                    f2_unpack(acc[0], a0, a1);
+                    f2_unpack(acc[1], a2, a3);
+                    f2_unpack(acc[2], a4, a5);
+                    f2_unpack(acc[3], a6, a7);
+                    l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(L::B_P_FULL + t));
