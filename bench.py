@@ -14,6 +14,10 @@ but the barrier and the max-over-ranks timing reduction (weak scaling).
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (the
 reference arm): each step is a bounded sample of the same workload.
+
+``--sweep`` instead prints one line per sequence length of the page's
+"Try It Yourself" sweep (B=1, H=32, d=128, causal, N = 512..8192), device
+timed like the main line; it is an extra curve, not the headline number.
 """
 
 from __future__ import annotations
@@ -424,6 +428,48 @@ def run_ours(args, w):
     return 0
 
 
+def run_sweep(args):
+    import torch
+
+    import exact_attention_122_b200 as fa
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device=dev)
+    peak, _, peak_src = load_peaks()
+    for N in synth.SWEEP_SEQ_LENS:
+        w = synth.sweep_workload(N)
+        q, k, v = (t.to(dev) for t in synth.workload_qkv(w))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        # at least ~200 ms of timed work per length, and at least args.steps launches
+        steps = max(args.steps, int(0.2 / max(w.flops / 1.0e15, 1e-6)))
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for _ in range(steps):
+                fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / steps
+        st, word = fa.device_status(stream.cuda_stream)
+        if st != fa.FA_OK:
+            raise SystemExit(f"kernel status {fa.status_string(st)} {word:#x}")
+        value = w.flops / (ms / 1e3) / 1e12
+        print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+                          "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
+                          "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                          "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                                     "causal": True},
+                          "pct_of_peak": 100.0 * value / peak, "peak_source": peak_src}),
+              flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,11 +481,15 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target length of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="print the sequence-length sweep curve instead of the headline line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.steps < 1:
         raise SystemExit("--steps must be >= 1")
+    if args.sweep:
+        return run_sweep(args)
     w = synth.workload(args.workload)
     if args.impl == "reference":
         return run_reference(args, w)

@@ -14,8 +14,8 @@ FA_ERR_LAUNCH = 4
 FA_ERR_TIMEOUT = 5
 FA_ERR_NO_DEVICE = 6
 
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_debug", "fa_get_device_status", "fa_status_string",
-                    "fa_last_cuda_error", "fa_version")
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_debug", "fa_get_device_status",
+                    "fa_status_string", "fa_last_cuda_error", "fa_version")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -39,6 +39,9 @@ def library() -> ctypes.CDLL:
     fwd_args = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
     lib.fa_fwd.argtypes = fwd_args
     lib.fa_fwd.restype = i
+    lib.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, ctypes.POINTER(ctypes.c_longlong),
+                                   i, f, vp]
+    lib.fa_fwd_strided.restype = i
     lib.fa_fwd_debug.argtypes = fwd_args + [u, i]
     lib.fa_fwd_debug.restype = i
     lib.fa_get_device_status.argtypes = [vp, ctypes.POINTER(u)]
@@ -78,6 +81,16 @@ def fa_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: 
                             stream_ptr)
 
 
+def fa_fwd_strided_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int,
+                       H: int, N: int, d: int, strides, causal: int, scale: float,
+                       stream_ptr: int) -> int:
+    """Direct call of fa_fwd_strided; ``strides`` = 12 element strides
+    (batch, head, seq) of q, k, v, o.  Returns the fa_status code."""
+    arr = (ctypes.c_longlong * 12)(*[int(x) for x in strides])
+    return library().fa_fwd_strided(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, arr, causal,
+                                    scale, stream_ptr)
+
+
 def fa_fwd_debug_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal, scale, stream_ptr,
                      watchdog_ms: int, inject: int) -> int:
     return library().fa_fwd_debug(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal, scale,
@@ -95,32 +108,41 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, 
            stream=None):
     """O, LSE = exact attention forward of bf16 (B, H, N, d) CUDA tensors.
 
-    ``out`` (bf16, same shape) and ``lse`` (float32, (B, H, N)) are allocated
-    with torch when not given.  Runs asynchronously on ``stream`` (default:
-    the current torch stream of q's device).
+    q, k, v and ``out`` may be strided views (for example a (B, N, H, d)
+    tensor transposed to (B, H, N, d)) as long as the head dimension is
+    contiguous; ``out`` (bf16) is allocated contiguous when not given and
+    ``lse`` (float32, contiguous (B, H, N)) likewise.  Runs asynchronously on
+    ``stream`` (default: the current torch stream of q's device).
     """
     import torch
 
     for name, t in (("q", q), ("k", k), ("v", v)):
-        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()):
-            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor of shape (B, H, N, d)")
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.stride(-1) == 1):
+            raise ValueError(f"{name} must be a bf16 CUDA tensor of shape (B, H, N, d) with a "
+                             "contiguous last dimension")
     if k.shape != q.shape or v.shape != q.shape or k.device != q.device or v.device != q.device:
         raise ValueError("q, k, v must share shape and device")
     B, H, N, d = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if not (out.is_cuda and out.dtype == torch.bfloat16 and out.shape == q.shape and out.is_contiguous()):
-        raise ValueError("out must be a contiguous bf16 CUDA tensor shaped like q")
+    if not (out.is_cuda and out.dtype == torch.bfloat16 and out.shape == q.shape and out.stride(-1) == 1):
+        raise ValueError("out must be a bf16 CUDA tensor shaped like q with a contiguous last dimension")
     if not (lse.is_cuda and lse.dtype == torch.float32 and tuple(lse.shape) == (B, H, N) and lse.is_contiguous()):
         raise ValueError("lse must be a contiguous float32 CUDA tensor of shape (B, H, N)")
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
-        st = fa_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                        B, H, N, d, 1 if causal else 0, float(scale), s.cuda_stream)
+        if all(t.is_contiguous() for t in (q, k, v, out)):
+            st = fa_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                            B, H, N, d, 1 if causal else 0, float(scale), s.cuda_stream)
+        else:
+            strides = [x for t in (q, k, v, out) for x in t.stride()[:3]]
+            st = fa_fwd_strided_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr(), B, H, N, d, strides, 1 if causal else 0,
+                                    float(scale), s.cuda_stream)
     if st != FA_OK:
         raise FaError(st)
     return out, lse

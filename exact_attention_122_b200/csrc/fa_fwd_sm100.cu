@@ -184,14 +184,14 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Watchd
     }
 }
 
-// TMA: 3-D tiled load (d offset, row, batch*head) into shared memory,
-// completing `bytes` on the mbarrier.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            int z, uint32_t bar) {
+// TMA: 4-D tiled load (d offset, row, head, batch) into shared memory,
+// completing its bytes on the mbarrier.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, int w, uint32_t bar) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
         : "memory");
 }
 
@@ -522,8 +522,9 @@ template <int D, int NS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ Og,
-                  float* __restrict__ LSEg, int BH, int N, int causal, float scale_log2,
-                  int hg, unsigned long long watchdog_ns, int inject) {
+                  float* __restrict__ LSEg, int BH, int H, int N, int causal, float scale_log2,
+                  int hg, long long o_sb, long long o_sh, long long o_sn,
+                  unsigned long long watchdog_ns, int inject) {
     using L = Layout<D, NS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -592,6 +593,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int kq = 0, u; (u = unit_index(kq, blockIdx.x, gridDim.x)) < num_units && ok;
                  ++kq, ++units) {
                 const Unit w = decode_unit(u, BH, N, causal, hg);
+                const int wb = w.bh / H, wh = w.bh - (w.bh / H) * H;   // batch, head
                 if (!wait_phase(bar(L::B_Q_EMPTY), (units & 1u) ^ 1u, wd, ROLE_PRODUCER, u)) {
                     ok = false;
                     break;
@@ -599,8 +601,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 mbar_arrive_expect_tx(bar(L::B_Q_FULL), 2 * L::Q_BYTES);
                 for (int t = 0; t < 2; ++t)
                     for (int h = 0; h < D / SW_COLS; ++h)
-                        tma_load_3d(sQ + t * L::Q_BYTES + h * L::HALF_BYTES, &tmQ, h * SW_COLS,
-                                    w.r0 + t * BM, w.bh, bar(L::B_Q_FULL));
+                        tma_load_4d(sQ + t * L::Q_BYTES + h * L::HALF_BYTES, &tmQ, h * SW_COLS,
+                                    w.r0 + t * BM, wh, wb, bar(L::B_Q_FULL));
                 ++q_issued;
                 for (int j = 0; j < w.nb1 && ok; ++j) {
                     for (int kind = 0; kind < 2; ++kind) {
@@ -617,8 +619,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             mbar_arrive_expect_tx(bar(L::B_KV_FULL + s), L::KV_BYTES);
                             const CUtensorMap* map = kind == 0 ? &tmK : &tmV;
                             for (int h = 0; h < D / SW_COLS; ++h)
-                                tma_load_3d(sKV + s * L::KV_BYTES + h * L::HALF_BYTES, map,
-                                            h * SW_COLS, j * BN, w.bh, bar(L::B_KV_FULL + s));
+                                tma_load_4d(sKV + s * L::KV_BYTES + h * L::HALF_BYTES, map,
+                                            h * SW_COLS, j * BN, wh, wb, bar(L::B_KV_FULL + s));
                         }
                         ++fills;
                     }
@@ -858,7 +860,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const float inv_l = 1.f / l;
             const bool store = row < N;
-            __nv_bfloat16* orow = Og + (size_t(w.bh) * N + (store ? row : 0)) * D;
+            const int wb = w.bh / H, wh = w.bh - (w.bh / H) * H;     // batch, head
+            __nv_bfloat16* orow = Og + wb * o_sb + wh * o_sh + (long long)(store ? row : 0) * o_sn;
             uint32_t ro[D];
             if constexpr (D == 128) {
                 tmem_ld128(tO, ro);
@@ -934,12 +937,20 @@ int Instance<D, NS>::regs[MAX_DEVICES];
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-fa_status encode_map(CUtensorMap* map, const void* base, int d, int N, long long BH) {
-    const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
-    const cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(d) * 2 * cuuint64_t(N)};
-    const cuuint32_t box[3] = {cuuint32_t(fa::SW_COLS), cuuint32_t(fa::BM), 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+// Element strides (batch, head, sequence) of one bf16 [B][H][N][d] operand;
+// the head dimension is always contiguous.
+struct Strides3 {
+    long long b, h, n;
+};
+
+// 4-D tensor map (d, N, H, B) with a (64, 128, 1, 1) box and 128-byte swizzle.
+fa_status encode_map(CUtensorMap* map, const void* base, int d, int N, int H, int B,
+                     const Strides3& st) {
+    const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(H), cuuint64_t(B)};
+    const cuuint64_t strides[3] = {cuuint64_t(st.n) * 2, cuuint64_t(st.h) * 2, cuuint64_t(st.b) * 2};
+    const cuuint32_t box[4] = {cuuint32_t(fa::SW_COLS), cuuint32_t(fa::BM), 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -948,8 +959,8 @@ fa_status encode_map(CUtensorMap* map, const void* base, int d, int N, long long
 
 template <int D, int NS>
 fa_status launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                 int N, int causal, float scale, cudaStream_t stream, int dev,
-                 unsigned long long watchdog_ns, int inject) {
+                 int N, const Strides3 (&st)[4], int causal, float scale, cudaStream_t stream,
+                 int dev, unsigned long long watchdog_ns, int inject) {
     using L = fa::Layout<D, NS>;
     auto kern = fa::fa_fwd_kernel<D, NS>;
     std::call_once(Instance<D, NS>::once[dev], [&] {
@@ -970,8 +981,9 @@ fa_status launch(const void* q, const void* k, const void* v, void* o, float* ls
     if (Instance<D, NS>::regs[dev] != fa::REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
     const long long BH = (long long)B * H;
     CUtensorMap mq, mk, mv;
-    if (encode_map(&mq, q, D, N, BH) != FA_OK || encode_map(&mk, k, D, N, BH) != FA_OK ||
-        encode_map(&mv, v, D, N, BH) != FA_OK)
+    if (encode_map(&mq, q, D, N, H, B, st[0]) != FA_OK ||
+        encode_map(&mk, k, D, N, H, B, st[1]) != FA_OK ||
+        encode_map(&mv, v, D, N, H, B, st[2]) != FA_OK)
         return FA_ERR_UNSUPPORTED;
     const long long nq2 = (N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
     const long long units = nq2 * BH;
@@ -989,8 +1001,9 @@ fa_status launch(const void* q, const void* k, const void* v, void* o, float* ls
     const int grid = int(units < g_dev[dev].sm_count ? units : g_dev[dev].sm_count);
     const float scale_log2 = scale * 1.4426950408889634f;
     kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o),
-                                                     lse, int(BH), N, causal, scale_log2,
-                                                     int(hg), watchdog_ns, inject);
+                                                     lse, int(BH), H, N, causal, scale_log2,
+                                                     int(hg), st[3].b, st[3].h, st[3].n,
+                                                     watchdog_ns, inject);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         t_last_cuda_error = int(e);
@@ -1000,8 +1013,8 @@ fa_status launch(const void* q, const void* k, const void* v, void* o, float* ls
 }
 
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                   int N, int d, int causal, float scale, void* stream, unsigned watchdog_ms,
-                   int inject) {
+                   int N, int d, const long long* strides12, int causal, float scale, void* stream,
+                   unsigned watchdog_ms, int inject) {
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
@@ -1011,6 +1024,27 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     if ((long long)B * H > 0x7fffffffLL || N > (1 << 30)) return FA_ERR_UNSUPPORTED;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
         return FA_ERR_MISALIGNED;
+    // Strides: q, k, v, o in that order, each (batch, head, sequence) in
+    // elements; NULL means contiguous [B][H][N][d].
+    Strides3 st[4];
+    for (int i = 0; i < 4; ++i) {
+        if (strides12) {
+            st[i] = Strides3{strides12[3 * i], strides12[3 * i + 1], strides12[3 * i + 2]};
+        } else {
+            st[i] = Strides3{(long long)H * N * d, (long long)N * d, (long long)d};
+        }
+        // The stride of a dimension of size 1 is never used; frameworks may
+        // report any value there, so it is replaced by a valid one.
+        if (B == 1) st[i].b = d;
+        if (H == 1) st[i].h = d;
+        if (N == 1) st[i].n = d;
+        const long long v3[3] = {st[i].b, st[i].h, st[i].n};
+        for (long long x : v3) {
+            if (x < d) return FA_ERR_INVALID_ARG;               // rows may not overlap within a head dim
+            if ((x * 2) % 16 != 0) return FA_ERR_MISALIGNED;   // TMA strides are multiples of 16 bytes
+            if (x * 2 >= (1LL << 40)) return FA_ERR_UNSUPPORTED;
+        }
+    }
 
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1041,8 +1075,9 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
 
     const unsigned long long wd_ns = (watchdog_ms ? watchdog_ms : 4000u) * 1000000ull;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (d == 64) return launch<64, 8>(q, k, v, o, lse, B, H, N, causal, scale, s, dev, wd_ns, inject);
-    return launch<128, 4>(q, k, v, o, lse, B, H, N, causal, scale, s, dev, wd_ns, inject);
+    if (d == 64)
+        return launch<64, 8>(q, k, v, o, lse, B, H, N, st, causal, scale, s, dev, wd_ns, inject);
+    return launch<128, 4>(q, k, v, o, lse, B, H, N, st, causal, scale, s, dev, wd_ns, inject);
 }
 
 }  // namespace
@@ -1051,13 +1086,21 @@ extern "C" {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int N, int d, int causal, float scale, void* stream) {
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, stream, 0, 0);
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, nullptr, causal, scale, stream, 0, 0);
+}
+
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int N, int d, const long long* strides, int causal, float scale,
+                         void* stream) {
+    if (!strides) return FA_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale, stream, 0, 0);
 }
 
 fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int H, int N, int d, int causal, float scale, void* stream,
                        unsigned watchdog_ms, int inject) {
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, stream, watchdog_ms, inject);
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, nullptr, causal, scale, stream, watchdog_ms,
+                    inject);
 }
 
 fa_status fa_get_device_status(void* stream, unsigned* detail) {

@@ -74,6 +74,26 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * fa_fwd_strided -- fa_fwd for strided operands, e.g. [B][N][H][d] tensors
+ * viewed as (B, H, N, d) (the layout transformer projections produce).
+ *
+ *  strides : 12 int64 values, element strides (batch, head, sequence) of q,
+ *            k, v and o in that order.  The head dimension d is always
+ *            contiguous.  Each stride must be >= d and a multiple of 8
+ *            elements (16 bytes, a TMA requirement), except that the stride
+ *            of a dimension of size 1 is ignored.  Rows of o must not
+ *            overlap and o must not overlap q, k, v or lse.
+ *  lse     : contiguous float [B][H][N] as in fa_fwd.
+ * Other arguments as fa_fwd.  Errors: FA_ERR_INVALID_ARG for a NULL
+ * `strides` or a stride < d, FA_ERR_MISALIGNED for a stride that is not a
+ * multiple of 8 elements, FA_ERR_UNSUPPORTED for a stride of 2^39 elements or
+ * more; otherwise as fa_fwd.
+ */
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int H, int N, int d, const long long* strides, int causal,
+                         float scale, void* stream);
+
+/*
  * fa_fwd_debug -- fa_fwd with the kernel watchdog exposed, for tests.
  *
  *  watchdog_ms : every wait inside the kernel gives up after this many

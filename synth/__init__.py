@@ -68,6 +68,17 @@ WORKLOADS = [
 ]
 
 
+# The sequence-length sweep of the "Try It Yourself" script on the page
+# "FlashAttention: The GPU Memory Hack That Changed Everything": batch 1,
+# 32 heads, head dim 128, causal, seq_len 512..8192 (the page uses fp16;
+# this path computes in bf16).
+SWEEP_SEQ_LENS = (512, 1024, 2048, 4096, 8192)
+
+
+def sweep_workload(N: int) -> Workload:
+    return Workload(100 + SWEEP_SEQ_LENS.index(N), f"seq_sweep_{N}", 1, 32, N, 128, True)
+
+
 def workload(index_or_name) -> Workload:
     for w in WORKLOADS:
         if w.index == index_or_name or w.name == index_or_name:

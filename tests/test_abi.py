@@ -83,3 +83,32 @@ def test_python_wrapper_rejects_cpu_tensors():
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fa.fa_fwd(q, q, q)
+
+
+def _contig(B, H, N, d):
+    return [H * N * d, N * d, d] * 4
+
+
+@pytest.mark.parametrize("mutate,expect", [
+    (lambda s: None, None),                                              # placeholder: NULL strides
+    (lambda s: s.__setitem__(2, 32), fa.FA_ERR_INVALID_ARG),            # q seq stride < d
+    (lambda s: s.__setitem__(5, 130), fa.FA_ERR_MISALIGNED),            # k seq stride not 8-aligned
+    (lambda s: s.__setitem__(9, 1 << 40), fa.FA_ERR_UNSUPPORTED),       # o batch stride too large
+    (lambda s: s.__setitem__(4, -128), fa.FA_ERR_INVALID_ARG),          # negative head stride
+])
+def test_strided_argument_validation(mutate, expect):
+    B, H, N, d = 2, 3, 8, 64
+    if expect is None:
+        lib = fa.library()
+        assert lib.fa_fwd_strided(P, P, P, P, P, B, H, N, d, None, 0, 1.0, 0) == fa.FA_ERR_INVALID_ARG
+        return
+    s = _contig(B, H, N, d)
+    mutate(s)
+    assert fa.fa_fwd_strided_raw(P, P, P, P, P, B, H, N, d, s, 0, 1.0, 0) == expect
+
+
+def test_strided_size_one_dims_ignore_their_strides():
+    # B = 1 and H = 1: any batch/head strides are accepted (they are never used);
+    # without a GPU the call then stops at the device query.
+    s = [1, 3, 64] * 4
+    assert fa.fa_fwd_strided_raw(P, P, P, P, P, 1, 1, 8, 64, s, 0, 1.0, 0) == fa.FA_ERR_NO_DEVICE

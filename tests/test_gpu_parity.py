@@ -261,3 +261,54 @@ def test_side_stream(fa):
         o, lse = run(fa, q, k, v, True, 1 / math.sqrt(128), stream=s)
     O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=True, scale=1 / math.sqrt(128))
     check(o, lse, O_ref, L_ref, "side stream")
+
+
+# ---------------------------------------------------------------------------
+# Strided operands (fa_fwd_strided)
+# ---------------------------------------------------------------------------
+def _bnhd(t):
+    """A (B, H, N, d) view of a contiguous (B, N, H, d) copy of t."""
+    return t.transpose(1, 2).contiguous().transpose(1, 2)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d,N", [(64, 300), (128, 513), (128, 1024)])
+def test_bnhd_views(fa, d, N, causal):
+    B, H = 2, 3
+    q, k, v = synth.draw_qkv(B, H, N, d, seed=400 + N + d + int(causal))
+    qd, kd, vd = (_bnhd(t).to("cuda:0") for t in (q, k, v))
+    assert not qd.is_contiguous()
+    out = torch.empty(B, N, H, d, dtype=torch.bfloat16, device="cuda:0").transpose(1, 2)
+    o, lse = fa.fa_fwd(qd, kd, vd, causal=causal, out=out)
+    torch.cuda.synchronize()
+    assert o.data_ptr() == out.data_ptr()
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=causal, scale=1 / math.sqrt(d))
+    check(o, lse, O_ref, L_ref, f"BNHD d={d} N={N} causal={causal}")
+
+
+def test_padded_and_mixed_strides(fa):
+    B, H, N, d = 2, 2, 700, 128
+    q, k, v = synth.draw_qkv(B, H, N, d, seed=91)
+    qpad = torch.zeros(B, H, N, d + 64, dtype=torch.bfloat16)
+    qpad[..., :d] = q
+    qd = qpad.to("cuda:0")[..., :d]                       # sequence stride d + 64
+    kd = _bnhd(k).to("cuda:0")                            # BNHD
+    vd = v.to("cuda:0")                                   # contiguous
+    opad = torch.full((B, H, N + 5, d + 8), float("nan"), dtype=torch.bfloat16, device="cuda:0")
+    out = opad[:, :, :N, :d]                              # padded output rows
+    o, lse = fa.fa_fwd(qd, kd, vd, causal=True, out=out)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=True, scale=1 / math.sqrt(d))
+    check(o, lse, O_ref, L_ref, "padded/mixed strides")
+    # nothing written outside the view
+    assert bool(torch.isnan(opad[:, :, N:, :]).all()) and bool(torch.isnan(opad[..., d:]).all())
+
+
+def test_strided_matches_contiguous_bitwise(fa):
+    B, H, N, d = 1, 4, 640, 128
+    q, k, v = synth.draw_qkv(B, H, N, d, seed=17)
+    o1, l1 = run(fa, q, k, v, True, 1 / math.sqrt(d))
+    qd, kd, vd = (_bnhd(t).to("cuda:0") for t in (q, k, v))
+    o2, l2 = fa.fa_fwd(qd, kd, vd, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
