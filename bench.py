@@ -3,7 +3,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one exact-attention forward (one fa_fwd launch) over one batch of
+A step is one exact-attention forward (one fa_fwd_dynamic launch, or fa_fwd
+with --schedule static) over one batch of
 the long-context causal workload (B=2, H=32, N=8192, d=128, bf16, seeded
 N(0,1) inputs), inputs resident in HBM.  FLOPs per step: 4*B*H*N^2*d / 2.
 Prints one JSON line (rank 0).
@@ -282,7 +283,7 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, args.gpus),
+        "config": workload_config(w, args.gpus, args.schedule),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -291,8 +292,9 @@ def run_reference(args, w):
     return 0
 
 
-def workload_config(w: synth.Workload, n_gpus: int):
-    return {"workload": w.name, "B_per_gpu": w.B, "H": w.H, "N": w.N, "d": w.d,
+def workload_config(w: synth.Workload, n_gpus: int, schedule: str = "dynamic"):
+    return {"workload": w.name, "schedule": schedule,
+            "B_per_gpu": w.B, "H": w.H, "N": w.N, "d": w.d,
             "causal": w.causal, "scale": w.scale, "global_batch": w.B * n_gpus, "seq_len": w.N,
             "parallelism": f"independent batches x{n_gpus}" if n_gpus > 1 else "single GPU",
             "l2": f"inputs {3 * w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB > 126 MB L2; no flush"}
@@ -324,7 +326,8 @@ def run_ours(args, w):
     stream = torch.cuda.Stream(device=dev)
 
     def step():
-        fa.fa_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=od, lse=lsed, stream=stream)
+        fa.fa_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=od, lse=lsed, stream=stream,
+                  schedule=args.schedule)
 
     def sync_all():
         torch.cuda.synchronize(dev)
@@ -378,7 +381,8 @@ def run_ours(args, w):
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
-        fa.fa_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=od, lse=lsed, stream=stream)
+        fa.fa_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=od, lse=lsed, stream=stream,
+                  schedule=args.schedule)
         oh.copy_(od, non_blocking=True)
         lh.copy_(lsed, non_blocking=True)
 
@@ -404,7 +408,7 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w, world),
+        "config": workload_config(w, world, args.schedule),
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": traffic,
@@ -446,13 +450,15 @@ def run_sweep(args):
         steps = max(args.steps, int(0.2 / max(w.flops / 1.0e15, 1e-6)))
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
-                fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream)
+                fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream,
+                          schedule=args.schedule)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize(dev)
             e0.record(stream)
             for _ in range(steps):
-                fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream)
+                fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream,
+                          schedule=args.schedule)
             e1.record(stream)
         torch.cuda.synchronize(dev)
         ms = e0.elapsed_time(e1) / steps
@@ -464,7 +470,7 @@ def run_sweep(args):
                           "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
                           "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
                           "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                                     "causal": True},
+                                     "causal": True, "schedule": args.schedule},
                           "pct_of_peak": 100.0 * value / peak, "peak_source": peak_src}),
               flush=True)
     return 0
@@ -481,6 +487,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target length of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--schedule", choices=["static", "dynamic"], default="dynamic",
+                    help="work distribution: fa_fwd_dynamic (default; measured 3-5 %% faster "
+                         "on the long causal workloads) or fa_fwd (static)")
     ap.add_argument("--sweep", action="store_true",
                     help="print the sequence-length sweep curve instead of the headline line")
     args = ap.parse_args(argv)

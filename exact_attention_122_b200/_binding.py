@@ -14,8 +14,9 @@ FA_ERR_LAUNCH = 4
 FA_ERR_TIMEOUT = 5
 FA_ERR_NO_DEVICE = 6
 
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_debug", "fa_get_device_status",
-                    "fa_status_string", "fa_last_cuda_error", "fa_version")
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_debug",
+                    "fa_get_device_status", "fa_status_string", "fa_last_cuda_error", "fa_version")
+DYNAMIC_WORKSPACE_BYTES = 256          # FA_DYNAMIC_WORKSPACE_BYTES in include/fa.h
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -42,6 +43,9 @@ def library() -> ctypes.CDLL:
     lib.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, ctypes.POINTER(ctypes.c_longlong),
                                    i, f, vp]
     lib.fa_fwd_strided.restype = i
+    lib.fa_fwd_dynamic.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, ctypes.POINTER(ctypes.c_longlong),
+                                   i, f, vp, ctypes.c_size_t, vp]
+    lib.fa_fwd_dynamic.restype = i
     lib.fa_fwd_debug.argtypes = fwd_args + [u, i]
     lib.fa_fwd_debug.restype = i
     lib.fa_get_device_status.argtypes = [vp, ctypes.POINTER(u)]
@@ -91,6 +95,31 @@ def fa_fwd_strided_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: 
                                     scale, stream_ptr)
 
 
+def fa_fwd_dynamic_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int,
+                       H: int, N: int, d: int, strides, causal: int, scale: float, ws_ptr: int,
+                       ws_bytes: int, stream_ptr: int) -> int:
+    """Direct call of fa_fwd_dynamic; ``strides`` = None or 12 element strides."""
+    arr = None if strides is None else (ctypes.c_longlong * 12)(*[int(x) for x in strides])
+    return library().fa_fwd_dynamic(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, arr, causal,
+                                    scale, ws_ptr, ws_bytes, stream_ptr)
+
+
+_WORKSPACES = {}
+
+
+def _workspace(device, stream):
+    """A DYNAMIC_WORKSPACE_BYTES device buffer per (device, stream): calls on one
+    stream are ordered, so they can share it."""
+    import torch
+
+    key = (str(device), int(stream.cuda_stream))
+    ws = _WORKSPACES.get(key)
+    if ws is None:
+        ws = torch.empty(DYNAMIC_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+        _WORKSPACES[key] = ws
+    return ws
+
+
 def fa_fwd_debug_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal, scale, stream_ptr,
                      watchdog_ms: int, inject: int) -> int:
     return library().fa_fwd_debug(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal, scale,
@@ -105,7 +134,7 @@ def device_status(stream_ptr: int = 0):
 
 
 def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-           stream=None):
+           stream=None, schedule: str = "static", workspace=None):
     """O, LSE = exact attention forward of bf16 (B, H, N, d) CUDA tensors.
 
     q, k, v and ``out`` may be strided views (for example a (B, N, H, d)
@@ -113,6 +142,9 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, 
     contiguous; ``out`` (bf16) is allocated contiguous when not given and
     ``lse`` (float32, contiguous (B, H, N)) likewise.  Runs asynchronously on
     ``stream`` (default: the current torch stream of q's device).
+    ``schedule="dynamic"`` uses fa_fwd_dynamic with ``workspace`` (a device
+    tensor of at least DYNAMIC_WORKSPACE_BYTES bytes; one cached per stream
+    when not given).
     """
     import torch
 
@@ -133,9 +165,19 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, 
         raise ValueError("out must be a bf16 CUDA tensor shaped like q with a contiguous last dimension")
     if not (lse.is_cuda and lse.dtype == torch.float32 and tuple(lse.shape) == (B, H, N) and lse.is_contiguous()):
         raise ValueError("lse must be a contiguous float32 CUDA tensor of shape (B, H, N)")
+    if schedule not in ("static", "dynamic"):
+        raise ValueError("schedule must be 'static' or 'dynamic'")
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
-        if all(t.is_contiguous() for t in (q, k, v, out)):
+        contiguous = all(t.is_contiguous() for t in (q, k, v, out))
+        if schedule == "dynamic":
+            ws = workspace if workspace is not None else _workspace(q.device, s)
+            strides = None if contiguous else [x for t in (q, k, v, out) for x in t.stride()[:3]]
+            st = fa_fwd_dynamic_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr(), B, H, N, d, strides, 1 if causal else 0,
+                                    float(scale), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                    s.cuda_stream)
+        elif contiguous:
             st = fa_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                             B, H, N, d, 1 if causal else 0, float(scale), s.cuda_stream)
         else:

@@ -44,7 +44,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "fa.h"
 
@@ -108,9 +110,13 @@ struct Layout {
     static constexpr int B_O_FULL = 2 * NS + 6;      // [2]
     static constexpr int B_O_EMPTY = 2 * NS + 8;     // [2]
     static constexpr int B_DRAIN = 2 * NS + 10;
-    static constexpr int NUM_BARS = 2 * NS + 11;
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem base, abort flag
-    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int B_UFULL = 2 * NS + 11;      // [2] unit queue (dynamic schedule)
+    static constexpr int B_UEMPTY = 2 * NS + 13;     // [2]
+    static constexpr int NUM_BARS = 2 * NS + 15;
+    // tmem base, abort flag, zero flag, spare, unit queue slots [2]
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int OFF_UNIT = OFF_MISC + 16;
+    static constexpr int BYTES = OFF_MISC + 32;
     static constexpr int ALLOC = BYTES + 1024;       // slack to align the base to 1 KiB
     // TMEM columns
     static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
@@ -523,7 +529,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ Og,
                   float* __restrict__ LSEg, int BH, int H, int N, int causal, float scale_log2,
-                  int hg, long long o_sb, long long o_sh, long long o_sn,
+                  int hg, long long o_sb, long long o_sh, long long o_sn, int* __restrict__ sched,
                   unsigned long long watchdog_ns, int inject) {
     using L = Layout<D, NS>;
     extern __shared__ uint8_t smem_raw[];
@@ -538,6 +544,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // Always 0: the abort flag of the drain waits, which must not be cut
     // short by the CTA's own abort.
     volatile int* zero_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);
+    volatile int* unit_slot = reinterpret_cast<volatile int*>(smem + L::OFF_UNIT);
     auto bar = [&](int i) { return sBar + 8u * uint32_t(i); };
 
     const int warp = threadIdx.x >> 5;
@@ -545,6 +552,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int nq2 = (N + UNIT_ROWS - 1) / UNIT_ROWS;
     const int num_units = nq2 * BH;
     const int nkb = (N + BN - 1) / BN;
+    const Watchdog wd_in{abort_flag, watchdog_ns};
+    // Unit queue.  Static schedule (sched == nullptr): every role walks the
+    // same boustrophedon sequence.  Dynamic schedule: the producer claims
+    // sequence indices from the global counter *sched and publishes them in
+    // two shared-memory slots (full: producer; empty: MMA thread and every
+    // softmax thread); -1 ends the CTA's work.
+    auto next_unit_consumer = [&](int kq, bool& ok_out, uint32_t role) -> int {
+        if (!sched) {
+            const int u = unit_index(kq, blockIdx.x, gridDim.x);
+            return u < num_units ? u : -1;
+        }
+        const int slot = kq & 1;
+        bool got = wait_phase(bar(L::B_UFULL + slot), uint32_t(kq >> 1) & 1u, wd_in, role, 0);
+        if (role == ROLE_SOFTMAX) got = __all_sync(0xffffffffu, got);
+        if (!got) {
+            ok_out = false;
+            return -1;
+        }
+        const int u = unit_slot[slot];
+        mbar_arrive(bar(L::B_UEMPTY + slot));
+        return u;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -560,6 +589,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(bar(L::B_O_EMPTY + t), BM);
         }
         mbar_init(bar(L::B_DRAIN), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(L::B_UFULL + i), 1);
+            mbar_init(bar(L::B_UEMPTY + i), 1 + 2 * BM);   // MMA thread + softmax threads
+        }
         *abort_flag = 0;
         *zero_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -590,8 +623,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t fills = 0, units = 0, q_issued = 0;
             bool ok = true;
             bool skipped = false;           // fault injection: fill 0 was never issued
-            for (int kq = 0, u; (u = unit_index(kq, blockIdx.x, gridDim.x)) < num_units && ok;
-                 ++kq, ++units) {
+            for (int kq = 0; ok; ++kq, ++units) {
+                int u;
+                if (sched) {
+                    // claim the next unit and publish it to the other roles
+                    const int slot = kq & 1;
+                    if (!wait_phase(bar(L::B_UEMPTY + slot), (uint32_t(kq >> 1) & 1u) ^ 1u, wd,
+                                    ROLE_PRODUCER, 0)) {
+                        ok = false;
+                        break;
+                    }
+                    u = atomicAdd(sched, 1);
+                    if (u >= num_units) u = -1;
+                    unit_slot[slot] = u;
+                    mbar_arrive(bar(L::B_UFULL + slot));
+                } else {
+                    u = unit_index(kq, blockIdx.x, gridDim.x);
+                    if (u >= num_units) u = -1;
+                }
+                if (u < 0) break;
                 const Unit w = decode_unit(u, BH, N, causal, hg);
                 const int wb = w.bh / H, wh = w.bh - (w.bh / H) * H;   // batch, head
                 if (!wait_phase(bar(L::B_Q_EMPTY), (units & 1u) ^ 1u, wd, ROLE_PRODUCER, u)) {
@@ -665,8 +715,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t stage_step = uint32_t(L::KV_BYTES >> 4);
             const uint32_t tS0 = tmem + L::TM_S0, tS1 = tmem + L::TM_S1;
             const uint32_t tO0 = tmem + L::TM_O0, tO1 = tmem + L::TM_O1;
-            for (int kq = 0, u; (u = unit_index(kq, blockIdx.x, gridDim.x)) < num_units && ok;
-                 ++kq, ++units) {
+            for (int kq = 0; ok; ++kq, ++units) {
+                const int u = next_unit_consumer(kq, ok, ROLE_MMA);
+                if (u < 0) break;
                 const Unit w = decode_unit(u, BH, N, causal, hg);
                 if (!wait_phase(bar(L::B_Q_FULL), units & 1u, wd, ROLE_MMA, u)) { ok = false; break; }
                 uint32_t sK = cons % NS;
@@ -769,7 +820,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t tO = tmem + lane_base + (t == 0 ? L::TM_O0 : L::TM_O1);
         uint32_t scnt = 0, ocnt = 0;
         bool ok = true;
-        for (int kq = 0, u; (u = unit_index(kq, blockIdx.x, gridDim.x)) < num_units && ok; ++kq) {
+        for (int kq = 0; ok; ++kq) {
+            const int u = next_unit_consumer(kq, ok, ROLE_SOFTMAX);
+            if (u < 0) break;
             const Unit w = decode_unit(u, BH, N, causal, hg);
             const int a = w.r0 + t * BM;             // first row of this sub-tile
             const int row = a + wr;
@@ -957,10 +1010,93 @@ fa_status encode_map(CUtensorMap* map, const void* base, int d, int N, int H, in
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_UNSUPPORTED;
 }
 
+// Heads per scheduling group.  The kernel orders units in groups of `hg`
+// heads (longest causal row blocks first inside a group) and deals them to
+// CTAs in boustrophedon order (decode_unit / unit_index).  Small groups keep
+// the K/V that concurrently running CTAs stream resident in L2; large groups
+// balance the CTAs better.  This replays the kernel's assignment on the host
+// for hg = 1, 2, 4, ..., BH (K/V tiles per unit as the cost) and takes the
+// lowest  (max CTA load / mean CTA load) x (1 + L2 penalty), the penalty
+// growing with the group's K/V bytes: 0 up to 16 MiB, then 3 %, 6 %, 9 % and
+// 12 % past 16, 32, 64 and 128 MiB (calibrated on the 8K and 32K causal
+// workloads, where 2-head groups measured 4-7 % faster than 8- or all-head
+// groups).  Decisions are cached per shape.
+struct HgKey {
+    long long BH;
+    int N, D, causal, grid;
+    bool operator==(const HgKey& o) const {
+        return BH == o.BH && N == o.N && D == o.D && causal == o.causal && grid == o.grid;
+    }
+};
+std::mutex g_hg_mutex;
+HgKey g_hg_keys[64];
+long long g_hg_vals[64];
+int g_hg_count = 0;
+
+double snake_imbalance(long long BH, int N, int causal, long long hg, int grid) {
+    const long long nq2 = (N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+    const long long nkb = (N + fa::BN - 1) / fa::BN;
+    const long long units = nq2 * BH;
+    std::vector<long long> load(size_t(grid), 0);
+    const long long per_group = hg * nq2;
+    for (long long i = 0; i < units; ++i) {
+        const long long g = i / per_group;
+        const long long r = i - g * per_group;
+        const long long gh = std::min(hg, BH - g * hg);
+        const long long level = r / gh;
+        const long long r0 = (causal ? (nq2 - 1 - level) : level) * fa::UNIT_ROWS;
+        const long long nb0 = causal ? std::min(r0 / fa::BN + 1, nkb) : nkb;
+        const long long nb1 = causal ? std::min(r0 / fa::BN + 2, nkb) : nkb;
+        const long long k = i / grid, c = i - k * grid;
+        load[size_t((k & 1) ? (grid - 1 - c) : c)] += nb0 + nb1 + 2;   // +2: per-unit overhead
+    }
+    long long mx = 0, sum = 0;
+    for (long long x : load) {
+        mx = std::max(mx, x);
+        sum += x;
+    }
+    return double(mx) * grid / double(sum);
+}
+
+long long choose_head_group(long long BH, int N, int D, int causal, int grid) {
+    const HgKey key{BH, N, D, causal, grid};
+    {
+        std::lock_guard<std::mutex> lk(g_hg_mutex);
+        for (int i = 0; i < g_hg_count; ++i)
+            if (g_hg_keys[i] == key) return g_hg_vals[i];
+    }
+    const long long kv_head_bytes = 2LL * N * D * 2;
+    long long best = BH;
+    double best_cost = 1e30;
+    // Bound the replay work for very large problems: beyond ~4M units the
+    // assignment statistics no longer depend on hg, so all heads form one group.
+    const long long units = ((N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS) * BH;
+    if (units <= (4LL << 20)) {
+        for (long long hg = 1;; hg = std::min(hg * 2, BH)) {
+            const double ws = double(hg * kv_head_bytes);
+            const double pen = ws <= 16.0 * (1 << 20) ? 0.0
+                             : ws <= 32.0 * (1 << 20) ? 0.03
+                             : ws <= 64.0 * (1 << 20) ? 0.06
+                             : ws <= 128.0 * (1 << 20) ? 0.09 : 0.12;
+            const double cost = snake_imbalance(BH, N, causal, hg, grid) * (1.0 + pen);
+            if (cost < best_cost - 1e-9) {
+                best_cost = cost;
+                best = hg;
+            }
+            if (hg == BH) break;
+        }
+    }
+    std::lock_guard<std::mutex> lk(g_hg_mutex);
+    const int slot = g_hg_count < 64 ? g_hg_count++ : int(BH % 64);
+    g_hg_keys[slot] = key;
+    g_hg_vals[slot] = best;
+    return best;
+}
+
 template <int D, int NS>
 fa_status launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                 int N, const Strides3 (&st)[4], int causal, float scale, cudaStream_t stream,
-                 int dev, unsigned long long watchdog_ns, int inject) {
+                 int N, const Strides3 (&st)[4], int causal, float scale, int* sched,
+                 cudaStream_t stream, int dev, unsigned long long watchdog_ns, int inject) {
     using L = fa::Layout<D, NS>;
     auto kern = fa::fa_fwd_kernel<D, NS>;
     std::call_once(Instance<D, NS>::once[dev], [&] {
@@ -987,22 +1123,29 @@ fa_status launch(const void* q, const void* k, const void* v, void* o, float* ls
         return FA_ERR_UNSUPPORTED;
     const long long nq2 = (N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
     const long long units = nq2 * BH;
-    // Heads per scheduling group.  When all of K and V fit in 32 MiB of L2
-    // there is nothing to group and the whole problem is one group (best
-    // balance); otherwise groups of two heads keep the K/V that concurrently
-    // running CTAs stream resident in L2 (measured best on the 8K and 32K
-    // causal workloads).
+    const int grid = int(units < g_dev[dev].sm_count ? units : g_dev[dev].sm_count);
+    // Static schedule: group size from the replayed assignment.  Dynamic
+    // schedule: CTAs claim units greedily, so balance no longer depends on the
+    // group size; groups then hold about 16 MiB of K/V (all heads when the
+    // whole K/V fits in 32 MiB).
     const long long kv_head_bytes = 2LL * N * D * 2;
-    long long hg = (BH * kv_head_bytes <= (32LL << 20)) ? BH : 2;
+    long long hg = sched ? ((BH * kv_head_bytes <= (32LL << 20)) ? BH : (16LL << 20) / kv_head_bytes)
+                         : choose_head_group(BH, N, D, causal, grid);
 #ifdef FA_HEAD_GROUP
     hg = FA_HEAD_GROUP;
 #endif
     hg = hg < 1 ? 1 : (hg > BH ? BH : hg);
-    const int grid = int(units < g_dev[dev].sm_count ? units : g_dev[dev].sm_count);
     const float scale_log2 = scale * 1.4426950408889634f;
+    if (sched) {
+        const cudaError_t me = cudaMemsetAsync(sched, 0, sizeof(int), stream);
+        if (me != cudaSuccess) {
+            t_last_cuda_error = int(me);
+            return FA_ERR_LAUNCH;
+        }
+    }
     kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o),
                                                      lse, int(BH), H, N, causal, scale_log2,
-                                                     int(hg), st[3].b, st[3].h, st[3].n,
+                                                     int(hg), st[3].b, st[3].h, st[3].n, sched,
                                                      watchdog_ns, inject);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
@@ -1013,8 +1156,8 @@ fa_status launch(const void* q, const void* k, const void* v, void* o, float* ls
 }
 
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                   int N, int d, const long long* strides12, int causal, float scale, void* stream,
-                   unsigned watchdog_ms, int inject) {
+                   int N, int d, const long long* strides12, int causal, float scale, int* sched,
+                   void* stream, unsigned watchdog_ms, int inject) {
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
@@ -1076,8 +1219,10 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     const unsigned long long wd_ns = (watchdog_ms ? watchdog_ms : 4000u) * 1000000ull;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (d == 64)
-        return launch<64, 8>(q, k, v, o, lse, B, H, N, st, causal, scale, s, dev, wd_ns, inject);
-    return launch<128, 4>(q, k, v, o, lse, B, H, N, st, causal, scale, s, dev, wd_ns, inject);
+        return launch<64, 8>(q, k, v, o, lse, B, H, N, st, causal, scale, sched, s, dev, wd_ns,
+                             inject);
+    return launch<128, 4>(q, k, v, o, lse, B, H, N, st, causal, scale, sched, s, dev, wd_ns,
+                          inject);
 }
 
 }  // namespace
@@ -1086,21 +1231,31 @@ extern "C" {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int N, int d, int causal, float scale, void* stream) {
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, nullptr, causal, scale, stream, 0, 0);
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, nullptr, causal, scale, nullptr, stream, 0, 0);
 }
 
 fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int H, int N, int d, const long long* strides, int causal, float scale,
                          void* stream) {
     if (!strides) return FA_ERR_INVALID_ARG;
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale, stream, 0, 0);
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale, nullptr, stream, 0, 0);
+}
+
+fa_status fa_fwd_dynamic(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int N, int d, const long long* strides, int causal, float scale,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace) return FA_ERR_INVALID_ARG;
+    if (workspace_bytes < FA_DYNAMIC_WORKSPACE_BYTES) return FA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return FA_ERR_MISALIGNED;
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale,
+                    static_cast<int*>(workspace), stream, 0, 0);
 }
 
 fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int H, int N, int d, int causal, float scale, void* stream,
                        unsigned watchdog_ms, int inject) {
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, nullptr, causal, scale, stream, watchdog_ms,
-                    inject);
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, nullptr, causal, scale, nullptr, stream,
+                    watchdog_ms, inject);
 }
 
 fa_status fa_get_device_status(void* stream, unsigned* detail) {

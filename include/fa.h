@@ -31,6 +31,8 @@
 #ifndef FA_B200_H
 #define FA_B200_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -92,6 +94,36 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
                          int B, int H, int N, int d, const long long* strides, int causal,
                          float scale, void* stream);
+
+/* Bytes of device workspace fa_fwd_dynamic needs (one work counter, padded). */
+#define FA_DYNAMIC_WORKSPACE_BYTES 256
+
+/*
+ * fa_fwd_dynamic -- fa_fwd / fa_fwd_strided with dynamic work distribution.
+ *
+ * The persistent CTAs claim 256-row units of work from a counter in
+ * `workspace` (longest causal rows first, heads grouped for L2 reuse)
+ * instead of following a fixed assignment, which balances the CTAs on
+ * shapes with few units per SM.  The result is identical to fa_fwd.  The
+ * parallel split over the sequence is the one of the page "FlashAttention:
+ * The GPU Memory Hack That Changed Everything", "FlashAttention-2: Even
+ * Faster".
+ *
+ *  strides         : NULL (contiguous [B][H][N][d]) or 12 strides as in
+ *                    fa_fwd_strided.
+ *  workspace       : device memory owned by the caller, 16-byte aligned,
+ *                    at least FA_DYNAMIC_WORKSPACE_BYTES bytes.  The call
+ *                    clears it on `stream` before the kernel runs, so its
+ *                    contents on entry do not matter; it must not be used
+ *                    by another call that may run at the same time.
+ *  workspace_bytes : its size.
+ * Other arguments as fa_fwd.  Errors: FA_ERR_INVALID_ARG for a NULL or too
+ * small workspace, FA_ERR_MISALIGNED for a misaligned one; otherwise as
+ * fa_fwd / fa_fwd_strided.
+ */
+fa_status fa_fwd_dynamic(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int H, int N, int d, const long long* strides, int causal,
+                         float scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * fa_fwd_debug -- fa_fwd with the kernel watchdog exposed, for tests.

@@ -112,3 +112,14 @@ def test_strided_size_one_dims_ignore_their_strides():
     # without a GPU the call then stops at the device query.
     s = [1, 3, 64] * 4
     assert fa.fa_fwd_strided_raw(P, P, P, P, P, 1, 1, 8, 64, s, 0, 1.0, 0) == fa.FA_ERR_NO_DEVICE
+
+
+def test_dynamic_argument_validation():
+    ws = 1 << 22
+    args = (P, P, P, P, P, 2, 3, 8, 64, None, 0, 1.0)
+    assert fa.fa_fwd_dynamic_raw(*args, 0, 256, 0) == fa.FA_ERR_INVALID_ARG          # NULL workspace
+    assert fa.fa_fwd_dynamic_raw(*args, ws, 255, 0) == fa.FA_ERR_INVALID_ARG         # too small
+    assert fa.fa_fwd_dynamic_raw(*args, ws + 4, 256, 0) == fa.FA_ERR_MISALIGNED      # misaligned
+    assert fa.DYNAMIC_WORKSPACE_BYTES == 256
+    text = open(HEADER).read()
+    assert "#define FA_DYNAMIC_WORKSPACE_BYTES 256" in text

@@ -312,3 +312,40 @@ def test_strided_matches_contiguous_bitwise(fa):
     o2, l2 = fa.fa_fwd(qd, kd, vd, causal=True)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ---------------------------------------------------------------------------
+# Dynamic work distribution (fa_fwd_dynamic): same arithmetic per unit, so
+# the result must equal the static schedule's bit for bit.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [(8, 12, 512, 64, False), (8, 12, 1024, 64, True),
+                                   (2, 3, 1000, 128, True), (2, 150, 256, 64, True),
+                                   (1, 32, 4096, 128, True)])
+def test_dynamic_equals_static(fa, shape):
+    B, H, N, d, causal = shape
+    q, k, v = synth.draw_qkv(B, H, N, d, seed=55 + N + H)
+    qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
+    o1, l1 = fa.fa_fwd(qd, kd, vd, causal=causal)
+    ws = torch.full((fa.DYNAMIC_WORKSPACE_BYTES,), 0x7f, dtype=torch.uint8, device="cuda:0")
+    for _ in range(2):                                    # dirty workspace, then reused
+        o2, l2 = fa.fa_fwd(qd, kd, vd, causal=causal, schedule="dynamic", workspace=ws)
+        torch.cuda.synchronize()
+        assert fa.device_status()[0] == fa.FA_OK
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    if N <= 1024:
+        O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=causal, scale=1 / math.sqrt(d))
+        check(o2, l2, O_ref, L_ref, f"dynamic {shape}")
+
+
+def test_dynamic_full_size_and_strided(fa):
+    w = synth.workload(4)
+    q, k, v = synth.workload_qkv(w)
+    qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
+    o1, l1 = fa.fa_fwd(qd, kd, vd, causal=True)
+    o2, l2 = fa.fa_fwd(qd, kd, vd, causal=True, schedule="dynamic")
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    qb, kb, vb = (_bnhd(t[:, :4]).to("cuda:0") for t in (q, k, v))   # 4 heads, BNHD views
+    o3, l3 = fa.fa_fwd(qb, kb, vb, causal=True, schedule="dynamic")
+    torch.cuda.synchronize()
+    assert torch.equal(o3, o1[:, :4]) and torch.equal(l3, l1[:, :4])
