@@ -1165,6 +1165,10 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     if (inject != 0 && inject != 1) return FA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if ((long long)B * H > 0x7fffffffLL || N > (1 << 30)) return FA_ERR_UNSUPPORTED;
+    // The kernel numbers 256-row units with 32-bit ints (and the dynamic
+    // schedule claims up to units + grid indices).
+    if (((long long)N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS * B * H > (1LL << 30))
+        return FA_ERR_UNSUPPORTED;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
         return FA_ERR_MISALIGNED;
     // Strides: q, k, v, o in that order, each (batch, head, sequence) in

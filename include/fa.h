@@ -61,7 +61,8 @@ typedef enum {
  *            backward pass that recomputes P ("Sizing a tile, and why the
  *            backward pass recomputes instead of storing").
  *  B, H, N : batch, heads, sequence length; each >= 1.  N need not be a
- *            multiple of the tile size.  B*H <= 2^31-1, N <= 2^30.
+ *            multiple of the tile size.  B*H <= 2^31-1, N <= 2^30, and
+ *            B*H*ceil(N/256) <= 2^30.
  *  d       : head dimension, 64 or 128 (else FA_ERR_UNSUPPORTED).
  *  causal  : 0 = no mask, 1 = key j allowed for query i iff j <= i.
  *  scale   : multiplier of Q K^T, finite and > 0 (usually 1/sqrt(d)).

@@ -123,3 +123,8 @@ def test_dynamic_argument_validation():
     assert fa.DYNAMIC_WORKSPACE_BYTES == 256
     text = open(HEADER).read()
     assert "#define FA_DYNAMIC_WORKSPACE_BYTES 256" in text
+
+
+def test_unit_count_limit():
+    # B*H*ceil(N/256) beyond 2^30 is refused before any device work.
+    assert fa.fa_fwd_raw(P, P, P, P, P, 1 << 12, 1 << 10, 1 << 17, 64, 0, 1.0, 0) == fa.FA_ERR_UNSUPPORTED
