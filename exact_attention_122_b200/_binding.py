@@ -14,8 +14,9 @@ FA_ERR_LAUNCH = 4
 FA_ERR_TIMEOUT = 5
 FA_ERR_NO_DEVICE = 6
 
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_debug",
-                    "fa_get_device_status", "fa_status_string", "fa_last_cuda_error", "fa_version")
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_dynamic_noalloc",
+                    "fa_fwd_debug", "fa_get_device_status", "fa_status_string",
+                    "fa_last_cuda_error", "fa_version")
 DYNAMIC_WORKSPACE_BYTES = 256          # FA_DYNAMIC_WORKSPACE_BYTES in include/fa.h
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -46,6 +47,9 @@ def library() -> ctypes.CDLL:
     lib.fa_fwd_dynamic.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, ctypes.POINTER(ctypes.c_longlong),
                                    i, f, vp, ctypes.c_size_t, vp]
     lib.fa_fwd_dynamic.restype = i
+    lib.fa_fwd_dynamic_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i,
+                                           ctypes.POINTER(ctypes.c_longlong), i, f, vp]
+    lib.fa_fwd_dynamic_noalloc.restype = i
     lib.fa_fwd_debug.argtypes = fwd_args + [u, i]
     lib.fa_fwd_debug.restype = i
     lib.fa_get_device_status.argtypes = [vp, ctypes.POINTER(u)]
@@ -102,6 +106,17 @@ def fa_fwd_dynamic_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: 
     arr = None if strides is None else (ctypes.c_longlong * 12)(*[int(x) for x in strides])
     return library().fa_fwd_dynamic(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, arr, causal,
                                     scale, ws_ptr, ws_bytes, stream_ptr)
+
+
+def fa_fwd_dynamic_noalloc_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int,
+                               B: int, H: int, N: int, d: int, strides, causal: int, scale: float,
+                               stream_ptr: int) -> int:
+    """Direct call of fa_fwd_dynamic_noalloc (no workspace: the library's
+    static device scratch holds the work counter).  ``strides`` = None or 12
+    element strides.  Returns the fa_status code."""
+    arr = None if strides is None else (ctypes.c_longlong * 12)(*[int(x) for x in strides])
+    return library().fa_fwd_dynamic_noalloc(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, arr,
+                                            causal, scale, stream_ptr)
 
 
 _WORKSPACES = {}

@@ -1231,6 +1231,36 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
 
 }  // namespace
 
+// ===========================================================================
+// Allocation-free variant of fa_fwd_dynamic (fa_fwd_dynamic_noalloc).
+//
+// Some callers cannot allocate device memory at all: a plugin loaded into an
+// application that owns every device allocation, or a latency-critical loop
+// that must not call cudaMalloc (it can synchronise the whole device).  For
+// them the dynamic schedule's work counter lives in this file-scope array
+// instead of a caller-provided workspace.  Every device that loads the
+// library holds these bytes from module load until the process exits.
+// ===========================================================================
+namespace fa {
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+static_assert(FA_DYNAMIC_WORKSPACE_BYTES <= FA_NOALLOC_SCRATCH_BYTES,
+              "the dynamic schedule's workspace must fit the static scratch");
+}  // namespace fa
+
+namespace {
+
+// Device address of g_noalloc_scratch, resolved once per device.  In host
+// code the array's name only stands for the device symbol: it is not a
+// device address and must never be handed to a kernel directly.
+struct NoallocScratch {
+    std::once_flag once;
+    cudaError_t err = cudaSuccess;
+    void* ptr = nullptr;
+};
+NoallocScratch g_noalloc[MAX_DEVICES];
+
+}  // namespace
+
 extern "C" {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -1253,6 +1283,34 @@ fa_status fa_fwd_dynamic(const void* q, const void* k, const void* v, void* o, f
     if (!aligned(workspace, 16)) return FA_ERR_MISALIGNED;
     return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale,
                     static_cast<int*>(workspace), stream, 0, 0);
+}
+
+fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int B, int H, int N, int d, const long long* strides, int causal,
+                                 float scale, void* stream) {
+    // The scratch holds one 32-bit counter of claimed units: problems with
+    // more units than it may count are refused before anything else.
+    if (B >= 1 && H >= 1 && N >= 1 &&
+        ((long long)N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS * B * H > FA_NOALLOC_MAX_UNITS)
+        return FA_ERR_UNSUPPORTED;
+    if (FA_DYNAMIC_WORKSPACE_BYTES > sizeof(fa::g_noalloc_scratch)) return FA_ERR_UNSUPPORTED;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
+        t_last_cuda_error = int(e);
+        return FA_ERR_NO_DEVICE;
+    }
+    // Set-up on the first call on this device (the device is current here).
+    NoallocScratch& ns = g_noalloc[dev];
+    std::call_once(ns.once, [&] { ns.err = cudaGetSymbolAddress(&ns.ptr, fa::g_noalloc_scratch); });
+    if (ns.err != cudaSuccess || ns.ptr == nullptr) {
+        t_last_cuda_error = int(ns.err);
+        return FA_ERR_LAUNCH;
+    }
+    // Same launch path as fa_fwd_dynamic: the counter is cleared on `stream`
+    // before the kernel runs.
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale,
+                    static_cast<int*>(ns.ptr), stream, 0, 0);
 }
 
 fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -126,6 +126,42 @@ fa_status fa_fwd_dynamic(const void* q, const void* k, const void* v, void* o, f
                          int B, int H, int N, int d, const long long* strides, int causal,
                          float scale, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of the library's static device scratch used by fa_fwd_dynamic_noalloc. */
+#define FA_NOALLOC_SCRATCH_BYTES 256
+/* Largest B*H*ceil(N/256) fa_fwd_dynamic_noalloc accepts (its counter's range). */
+#define FA_NOALLOC_MAX_UNITS (1LL << 30)
+
+/*
+ * fa_fwd_dynamic_noalloc -- fa_fwd_dynamic without a workspace argument, for
+ * callers that cannot allocate device memory (a plugin inside an
+ * application that owns every device allocation, or a latency-critical
+ * loop that must not call cudaMalloc, which can synchronise the device).
+ * The pages have no counterpart: this is a deployment variant, not part of
+ * the method.
+ *
+ * The dynamic schedule's work counter lives in a static device array of
+ * FA_NOALLOC_SCRATCH_BYTES bytes inside the library; every device that
+ * loads the library holds it until the process exits.  The call allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine); the
+ * caller still passes q, k, v, o and lse.
+ *
+ *  - The first call on a device resolves the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call shares the array and leaves its last contents there; the
+ *    call clears the counter on `stream` before its kernel runs.  Calls that
+ *    may overlap on the GPU (different streams not ordered by events) race
+ *    on the counter and give wrong results: serialise them.
+ *  - Problems with more than FA_NOALLOC_MAX_UNITS units (B*H*ceil(N/256))
+ *    exceed the counter's range and return FA_ERR_UNSUPPORTED.
+ *
+ * Arguments (strides NULL or 12 strides as in fa_fwd_strided), results and
+ * other errors as fa_fwd_dynamic; FA_ERR_LAUNCH if the set-up fails.
+ */
+fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int B, int H, int N, int d, const long long* strides, int causal,
+                                 float scale, void* stream);
+
 /*
  * fa_fwd_debug -- fa_fwd with the kernel watchdog exposed, for tests.
  *
