@@ -83,19 +83,34 @@ def softmax_rows_fp64(S: np.ndarray):
     return E / Z, M[:, 0], Z[:, 0]
 
 
-def attention_rows_fp64(q_bh, k_bh, v_bh, rows, causal: bool, scale: float):
+def attention_rows_fp64(q_bh, k_bh, v_bh, rows, causal: bool, scale: float,
+                        key_offset: int = 0):
     """O and LSE for selected query rows of one (batch, head).
 
-    q_bh, k_bh, v_bh: (N, d) float64.  rows: 1-D int array of query indices.
-    Materialises the full score rows S[rows, :] and P[rows, :] (all N keys),
-    then O = P V.  Returns (O (len(rows), d), LSE (len(rows),)).
+    q_bh: (N_q, d), k_bh, v_bh: (N_k, d) float64.  rows: 1-D int array of
+    query indices.  Materialises the full score rows S[rows, :] and P[rows, :]
+    (all N_k keys), then O = P V.  With causal masking query i may see key j
+    iff j <= i + key_offset (0 for square problems; N_k - N_q when the N_q
+    queries are the last N_q positions of the key sequence).  A row with no
+    allowed key gets O = 0 and LSE = -inf (the empty sum).
+    Returns (O (len(rows), d), LSE (len(rows),)).
     """
     rows = np.asarray(rows, dtype=np.int64)
     N = k_bh.shape[0]
     S = scale * (q_bh[rows] @ k_bh.T)                       # S = Q K^T * scale
     if causal:
         keys = np.arange(N, dtype=np.int64)
-        S = np.where(keys[None, :] <= rows[:, None], S, -np.inf)   # allowed iff j <= i
+        allowed = keys[None, :] <= rows[:, None] + key_offset
+        S = np.where(allowed, S, -np.inf)                   # allowed iff j <= i (+ offset)
+        empty = ~allowed.any(axis=1)
+        if empty.any():
+            O = np.zeros((len(rows), v_bh.shape[1]))
+            LSE = np.full(len(rows), -np.inf)
+            keep = ~empty
+            if keep.any():
+                O[keep], LSE[keep] = attention_rows_fp64(q_bh, k_bh, v_bh, rows[keep], causal,
+                                                         scale, key_offset)
+            return O, LSE
     P, M, Z = softmax_rows_fp64(S)                          # P = softmax(S)
     O = P @ v_bh                                            # O = P V
     LSE = M + np.log(Z)
@@ -104,16 +119,25 @@ def attention_rows_fp64(q_bh, k_bh, v_bh, rows, causal: bool, scale: float):
 
 def attention_fp64(q, k, v, causal: bool = False, scale: float | None = None,
                    row_chunk: int = 512):
-    """Exact attention forward in float64 for (B, H, N, d) inputs.
+    """Exact attention forward in float64: q (B, H, N_q, d), k and v
+    (B, H, N_k, d) (N_q = N_k for the square problems).
 
     Materialises S and P one chunk of ``row_chunk`` query rows at a time (rows
     are independent, so chunking changes no result; it bounds host memory for
-    N = 32768).  Returns (O (B,H,N,d) float64, LSE (B,H,N) float64).
+    N = 32768).  Causal masking when N_q < N_k treats the queries as the last
+    N_q positions: query i may see key j iff j <= i + N_k - N_q.
+    Returns (O (B,H,N_q,d) float64, LSE (B,H,N_q) float64).
     """
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
-    if q.ndim != 4 or k.shape != q.shape or v.shape != q.shape:
-        raise ValueError("q, k, v must share one (B, H, N, d) shape")
+    if q.ndim != 4 or k.ndim != 4 or v.shape != k.shape or q.shape[:2] != k.shape[:2] \
+            or q.shape[3] != k.shape[3]:
+        raise ValueError("q must be (B, H, N_q, d) and k, v (B, H, N_k, d)")
     B, H, N, d = q.shape
+    Nk = k.shape[2]
+    # N_q queries are the last N_q positions of the N_k keys (causal offset).
+    key_offset = Nk - N
+    if causal and key_offset < 0:
+        raise ValueError("causal attention needs N_q <= N_k")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     O = np.empty((B, H, N, d), dtype=np.float64)
@@ -124,7 +148,7 @@ def attention_fp64(q, k, v, causal: bool = False, scale: float | None = None,
                 r1 = min(N, r0 + row_chunk)
                 rows = np.arange(r0, r1)
                 O[b, h, r0:r1], LSE[b, h, r0:r1] = attention_rows_fp64(
-                    q[b, h], k[b, h], v[b, h], rows, causal, scale)
+                    q[b, h], k[b, h], v[b, h], rows, causal, scale, key_offset)
     return O, LSE
 
 

@@ -228,9 +228,67 @@ def pin_library_routine(seed=19):
             assert np.max(np.abs(LSE - scipy.special.logsumexp(S, axis=-1))) <= 1e-12
 
 
+def pin_decode_library(seed=23):
+    """N_q < N_k (queries = the last N_q positions): torch float64 SDPA with an
+    explicit lower-right boolean mask, and scipy logsumexp for LSE."""
+    rng = np.random.default_rng(seed)
+    for (Nq, Nk, d) in ((1, 37, 8), (5, 64, 16), (16, 300, 32)):
+        q = rng.standard_normal((2, 3, Nq, d)) * 2
+        k = rng.standard_normal((2, 3, Nk, d)) * 2
+        v = rng.standard_normal((2, 3, Nk, d))
+        scale = 1 / math.sqrt(d)
+        mask = np.tril(np.ones((Nq, Nk), bool), k=Nk - Nq)
+        for causal in (False, True):
+            O, LSE = oracle.attention_fp64(q, k, v, causal=causal, scale=scale)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v),
+                attn_mask=torch.from_numpy(mask) if causal else None, scale=scale).numpy()
+            assert np.max(np.abs(O - ref)) <= 1e-12
+            S = scale * np.einsum("bhid,bhjd->bhij", q, k)
+            if causal:
+                S = np.where(mask, S, -np.inf)
+            assert np.max(np.abs(LSE - scipy.special.logsumexp(S, axis=-1))) <= 1e-12
+
+
+def pin_decode_closed_form(seed=29):
+    """Equal scores with N_q < N_k: query i sees keys 0..i+N_k-N_q, so O_i is
+    their mean and LSE_i = ln(i + N_k - N_q + 1)."""
+    rng = np.random.default_rng(seed)
+    Nq, Nk, d = 4, 19, 8
+    q = np.zeros((1, 1, Nq, d))
+    k = rng.standard_normal((1, 1, Nk, d))
+    v = rng.standard_normal((1, 1, Nk, d))
+    O, LSE = oracle.attention_fp64(q, k, v, causal=True, scale=0.5)
+    for i in range(Nq):
+        cnt = i + Nk - Nq + 1
+        assert np.max(np.abs(O[0, 0, i] - v[0, 0, :cnt].mean(axis=0))) <= 1e-12
+        assert abs(LSE[0, 0, i] - math.log(cnt)) <= 1e-12
+
+
+def pin_decode_brute_force(seed=31):
+    """Tiny N_q < N_k case written out with scalar loops."""
+    rng = np.random.default_rng(seed)
+    Nq, Nk, d = 3, 7, 2
+    q = rng.standard_normal((1, 1, Nq, d))
+    k = rng.standard_normal((1, 1, Nk, d))
+    v = rng.standard_normal((1, 1, Nk, d))
+    scale = 0.7
+    O, LSE = oracle.attention_fp64(q, k, v, causal=True, scale=scale)
+    for i in range(Nq):
+        keys = [j for j in range(Nk) if j <= i + (Nk - Nq)]
+        sc = [scale * sum(q[0, 0, i, t] * k[0, 0, j, t] for t in range(d)) for j in keys]
+        mx = max(sc)
+        w = [math.exp(x - mx) for x in sc]
+        z = sum(w)
+        for t in range(d):
+            o = sum(wj * v[0, 0, j, t] for wj, j in zip(w, keys)) / z
+            assert abs(O[0, 0, i, t] - o) <= 1e-12
+        assert abs(LSE[0, 0, i] - (mx + math.log(z))) <= 1e-12
+
+
 PINS = [pin_worked_example_direct, pin_worked_example_tiled, pin_exercise1,
         pin_brute_force_tiling, pin_invariants, pin_closed_forms, pin_scale_handling,
-        pin_library_routine]
+        pin_library_routine, pin_decode_library, pin_decode_closed_form, pin_decode_brute_force]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -264,33 +322,33 @@ def test_rows_match_full():
 # Mutation tests: a plausible mistake planted in the oracle must fail a pin.
 # ---------------------------------------------------------------------------
 
-def _mut_causal_strict(q_bh, k_bh, v_bh, rows, causal, scale):
+def _mut_causal_strict(q_bh, k_bh, v_bh, rows, causal, scale, key_offset=0):
     rows = np.asarray(rows); N = k_bh.shape[0]
     S = scale * (q_bh[rows] @ k_bh.T)
     if causal:
-        S = np.where(np.arange(N)[None, :] < rows[:, None], S, -np.inf)   # j < i instead of j <= i
+        S = np.where(np.arange(N)[None, :] < rows[:, None] + key_offset, S, -np.inf)   # j < i, not j <= i
     P, M, Z = oa.softmax_rows_fp64(S)
     return P @ v_bh, M + np.log(Z)
 
 
-def _mut_no_scale(q_bh, k_bh, v_bh, rows, causal, scale):
-    return _ORIG_ROWS(q_bh, k_bh, v_bh, rows, causal, 1.0)                # scale dropped
+def _mut_no_scale(q_bh, k_bh, v_bh, rows, causal, scale, key_offset=0):
+    return _ORIG_ROWS(q_bh, k_bh, v_bh, rows, causal, 1.0, key_offset)    # scale dropped
 
 
-def _mut_lse_without_max(q_bh, k_bh, v_bh, rows, causal, scale):
+def _mut_lse_without_max(q_bh, k_bh, v_bh, rows, causal, scale, key_offset=0):
     rows = np.asarray(rows); N = k_bh.shape[0]
     S = scale * (q_bh[rows] @ k_bh.T)
     if causal:
-        S = np.where(np.arange(N)[None, :] <= rows[:, None], S, -np.inf)
+        S = np.where(np.arange(N)[None, :] <= rows[:, None] + key_offset, S, -np.inf)
     P, M, Z = oa.softmax_rows_fp64(S)
     return P @ v_bh, np.log(Z)                                            # M term dropped
 
 
-def _mut_transposed_keys(q_bh, k_bh, v_bh, rows, causal, scale):
+def _mut_transposed_keys(q_bh, k_bh, v_bh, rows, causal, scale, key_offset=0):
     rows = np.asarray(rows); N = k_bh.shape[0]
     S = scale * (q_bh[rows] @ k_bh[::-1].T)                               # key order reversed
     if causal:
-        S = np.where(np.arange(N)[None, :] <= rows[:, None], S, -np.inf)
+        S = np.where(np.arange(N)[None, :] <= rows[:, None] + key_offset, S, -np.inf)
     P, M, Z = oa.softmax_rows_fp64(S)
     return P @ v_bh, M + np.log(Z)
 
@@ -317,6 +375,10 @@ def _mut_blockmax_no_rescale(scores, values, block):
     return acc / l, m, l, trace
 
 
+def _mut_offset_ignored(q_bh, k_bh, v_bh, rows, causal, scale, key_offset=0):
+    return _ORIG_ROWS(q_bh, k_bh, v_bh, rows, causal, scale, 0)            # N_k - N_q dropped
+
+
 _ORIG_ROWS = oa.attention_rows_fp64
 
 MUTANTS = {
@@ -324,6 +386,7 @@ MUTANTS = {
     "no_scale": ("attention_rows_fp64", _mut_no_scale),
     "lse_without_max": ("attention_rows_fp64", _mut_lse_without_max),
     "transposed_keys": ("attention_rows_fp64", _mut_transposed_keys),
+    "offset_ignored": ("attention_rows_fp64", _mut_offset_ignored),
     "softmax_sign": ("softmax_rows_fp64", _mut_softmax_sign),
     "blockmax_no_rescale": ("online_softmax_row_blockmax", _mut_blockmax_no_rescale),
 }
