@@ -16,6 +16,10 @@ but the barrier and the max-over-ranks timing reduction (weak scaling).
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (the
 reference arm): each step is a bounded sample of the same workload.
 
+``--decode`` instead times the decode-shaped path (fa_fwd_decode: 1 new
+query per sequence against 32K keys, B=16, H=32, d=128), which is bound by
+reading K and V once: its metric is effective HBM GB/s.
+
 ``--sweep`` instead prints one line per sequence length of the page's
 "Try It Yourself" sweep (B=1, H=32, d=128, causal, N = 512..8192), device
 timed like the main line; it is an extra curve, not the headline number.
@@ -432,6 +436,58 @@ def run_ours(args, w):
     return 0
 
 
+def run_decode(args):
+    import torch
+
+    import exact_attention_122_b200 as fa
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = synth.DECODE_WORKLOAD
+    q, k, v = (t.to(dev) for t in synth.draw_decode_qkv(w.B, w.H, w.Nq, w.Nk, w.d, w.seed))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.decode_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        fa.fa_fwd_decode(q, k, v, causal=w.causal, out=o, lse=lse, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    gbs = w.algorithmic_bytes / (ms / 1e3) / 1e9
+    try:
+        with open(PEAKS_FILE) as f:
+            peak, src = float(json.load(f)["hbm_gbs"]), "measured hbm_gbs"
+    except (OSError, KeyError, ValueError):
+        peak, src = 6650.0, "fallback"
+    line = {"metric": "decode attention effective HBM GB/s (1 GPU)", "value": gbs, "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                       "causal": w.causal,
+                       "l2": f"K+V {w.kv_bytes / 1e9:.1f} GB > 126 MB L2; no flush"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                         "frac": gbs / peak, "traffic": None, "peak_source": src,
+                         "kernel": "decode_split_kernel + decode_merge_kernel"},
+            "gpu_launches": 2 * args.steps, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_sweep(args):
     import torch
 
@@ -490,6 +546,8 @@ def main(argv=None):
     ap.add_argument("--schedule", choices=["static", "dynamic"], default="dynamic",
                     help="work distribution: fa_fwd_dynamic (default; measured 3-5 %% faster "
                          "on the long causal workloads) or fa_fwd (static)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the decode-shaped path (HBM-bound) instead of the headline line")
     ap.add_argument("--sweep", action="store_true",
                     help="print the sequence-length sweep curve instead of the headline line")
     args = ap.parse_args(argv)
@@ -499,6 +557,8 @@ def main(argv=None):
         raise SystemExit("--steps must be >= 1")
     if args.sweep:
         return run_sweep(args)
+    if args.decode:
+        return run_decode(args)
     w = synth.workload(args.workload)
     if args.impl == "reference":
         return run_reference(args, w)

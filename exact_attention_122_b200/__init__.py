@@ -9,6 +9,7 @@ missing, importing the binding raises.
 from ._binding import (  # noqa: F401
     FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_MISALIGNED, FA_ERR_LAUNCH,
     FA_ERR_TIMEOUT, FA_ERR_NO_DEVICE, EXPORTED_SYMBOLS, DYNAMIC_WORKSPACE_BYTES,
+    DECODE_MAX_QUERIES, DECODE_MAX_SPLITS, decode_workspace_bytes, fa_fwd_decode, fa_fwd_decode_raw,
     FaError, library, library_path, status_string, version,
     fa_fwd, fa_fwd_raw, fa_fwd_strided_raw, fa_fwd_dynamic_raw, fa_fwd_dynamic_noalloc_raw,
     fa_fwd_debug_raw, device_status,

@@ -15,8 +15,10 @@ FA_ERR_TIMEOUT = 5
 FA_ERR_NO_DEVICE = 6
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_dynamic_noalloc",
-                    "fa_fwd_debug", "fa_get_device_status", "fa_status_string",
-                    "fa_last_cuda_error", "fa_version")
+                    "fa_fwd_decode_workspace_bytes", "fa_fwd_decode", "fa_fwd_debug",
+                    "fa_get_device_status", "fa_status_string", "fa_last_cuda_error", "fa_version")
+DECODE_MAX_QUERIES = 16                # FA_DECODE_MAX_QUERIES
+DECODE_MAX_SPLITS = 256                # FA_DECODE_MAX_SPLITS
 DYNAMIC_WORKSPACE_BYTES = 256          # FA_DYNAMIC_WORKSPACE_BYTES in include/fa.h
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -50,6 +52,10 @@ def library() -> ctypes.CDLL:
     lib.fa_fwd_dynamic_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i,
                                            ctypes.POINTER(ctypes.c_longlong), i, f, vp]
     lib.fa_fwd_dynamic_noalloc.restype = i
+    lib.fa_fwd_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    lib.fa_fwd_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_fwd_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, ctypes.c_size_t, vp]
+    lib.fa_fwd_decode.restype = i
     lib.fa_fwd_debug.argtypes = fwd_args + [u, i]
     lib.fa_fwd_debug.restype = i
     lib.fa_get_device_status.argtypes = [vp, ctypes.POINTER(u)]
@@ -117,6 +123,53 @@ def fa_fwd_dynamic_noalloc_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, l
     arr = None if strides is None else (ctypes.c_longlong * 12)(*[int(x) for x in strides])
     return library().fa_fwd_dynamic_noalloc(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, arr,
                                             causal, scale, stream_ptr)
+
+
+def decode_workspace_bytes(B: int, H: int, Nq: int, Nk: int, d: int, num_splits: int = 0) -> int:
+    return int(library().fa_fwd_decode_workspace_bytes(B, H, Nq, Nk, d, num_splits))
+
+
+def fa_fwd_decode_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int,
+                      Nq: int, Nk: int, d: int, causal: int, scale: float, num_splits: int,
+                      ws_ptr: int, ws_bytes: int, stream_ptr: int) -> int:
+    """Direct call of fa_fwd_decode; returns the fa_status code."""
+    return library().fa_fwd_decode(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, Nq, Nk, d, causal,
+                                   scale, num_splits, ws_ptr, ws_bytes, stream_ptr)
+
+
+def fa_fwd_decode(q, k, v, causal: bool = False, scale: float | None = None, num_splits: int = 0,
+                  out=None, lse=None, workspace=None, stream=None):
+    """O, LSE for few queries q (B, H, Nq, d) against k, v (B, H, Nk, d), bf16
+    contiguous CUDA tensors (Nq <= DECODE_MAX_QUERIES).  ``workspace`` (a
+    device tensor of at least decode_workspace_bytes(...) bytes) is allocated
+    with torch when not given."""
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if k.shape != (B, H, Nk, d) or v.shape != k.shape:
+        raise ValueError("k and v must be (B, H, Nk, d) with q's B, H, d")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(B, H, Nq, Nk, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        st = fa_fwd_decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr(), B, H, Nq, Nk, d, 1 if causal else 0, float(scale),
+                               int(num_splits), workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), s.cuda_stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_decode")
+    return out, lse
 
 
 _WORKSPACES = {}

@@ -11,8 +11,9 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SOURCES = [os.path.join(PKG, "csrc", "fa_fwd_sm100.cu")]
-HEADERS = [os.path.join(ROOT, "include", "fa.h")]
+SOURCES = [os.path.join(PKG, "csrc", "fa_fwd_sm100.cu"),
+           os.path.join(PKG, "csrc", "fa_decode_sm100.cu")]
+HEADERS = [os.path.join(ROOT, "include", "fa.h"), os.path.join(PKG, "csrc", "fa_internal.h")]
 LIB = os.path.join(PKG, "libfa_b200.so")
 
 NVCC_FLAGS = [
@@ -40,7 +41,8 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include")]
+    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
+           "-I", os.path.join(PKG, "csrc")]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     tmp = LIB + ".tmp"

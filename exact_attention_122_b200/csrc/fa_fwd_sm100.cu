@@ -49,6 +49,7 @@
 #include <vector>
 
 #include "fa.h"
+#include "fa_internal.h"
 
 namespace fa {
 
@@ -963,6 +964,12 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 thread_local int t_last_cuda_error = 0;
+
+}  // namespace
+
+void fa_internal::set_last_cuda_error(int e) { t_last_cuda_error = e; }
+
+namespace {
 
 constexpr int MAX_DEVICES = 64;
 struct DeviceInfo {

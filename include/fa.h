@@ -162,6 +162,50 @@ fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, vo
                                  int B, int H, int N, int d, const long long* strides, int causal,
                                  float scale, void* stream);
 
+/* Largest number of query rows per (batch, head) fa_fwd_decode accepts. */
+#define FA_DECODE_MAX_QUERIES 16
+/* Largest explicit split count of fa_fwd_decode. */
+#define FA_DECODE_MAX_SPLITS 256
+
+/*
+ * fa_fwd_decode_workspace_bytes -- device workspace fa_fwd_decode needs for
+ * these sizes (num_splits 0 = the automatic choice).  Returns 0 for sizes
+ * fa_fwd_decode would reject as invalid.
+ */
+size_t fa_fwd_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits);
+
+/*
+ * fa_fwd_decode -- exact attention for few queries against a long key
+ * sequence (decoding), split over the keys.
+ *
+ * Same operation as fa_fwd with separate lengths: q, o bf16 [B][H][Nq][d]
+ * and k, v bf16 [B][H][Nk][d], contiguous; lse float [B][H][Nq].  With
+ * causal = 1 the queries are the last Nq positions of the key sequence:
+ * query i may see key j iff j <= i + Nk - Nq (needs Nq <= Nk).  The keys
+ * are cut into `num_splits` ranges (0 = automatic) processed in parallel;
+ * each range keeps the online-softmax running state of the page "Flash
+ * attention optimization" ("The fix: tile the computation ..."), and a
+ * second kernel merges the ranges with that page's rescale-and-merge rule.
+ * This shape is bound by reading K and V once from device memory, so it
+ * runs on the CUDA cores.  P stays in fp32 here (no bf16 rounding of P).
+ *
+ *  Nq          : 1 .. FA_DECODE_MAX_QUERIES.
+ *  Nk          : >= 1 (>= Nq when causal), <= 2^30;  B*H <= 65535.
+ *  num_splits  : 0 (automatic) .. FA_DECODE_MAX_SPLITS.
+ *  workspace   : device memory owned by the caller, 256-byte aligned, at
+ *                least fa_fwd_decode_workspace_bytes(...) bytes; it holds
+ *                the per-split partial results and must not be shared by
+ *                calls that may run at the same time.
+ * Errors: FA_ERR_INVALID_ARG (NULL pointers or workspace, sizes < 1,
+ * causal with Nq > Nk, bad scale or split count, workspace too small),
+ * FA_ERR_UNSUPPORTED (d not 64/128, Nq > FA_DECODE_MAX_QUERIES, sizes beyond
+ * the limits, device not sm_100), FA_ERR_MISALIGNED, FA_ERR_NO_DEVICE,
+ * FA_ERR_LAUNCH.
+ */
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                        int num_splits, void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * fa_fwd_debug -- fa_fwd with the kernel watchdog exposed, for tests.
  *

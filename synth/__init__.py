@@ -79,6 +79,51 @@ def sweep_workload(N: int) -> Workload:
     return Workload(100 + SWEEP_SEQ_LENS.index(N), f"seq_sweep_{N}", 1, 32, N, 128, True)
 
 
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Few queries (the newest Nq positions) against Nk keys per (batch, head)."""
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def kv_bytes(self) -> int:
+        return 2 * self.B * self.H * self.Nk * self.d * 2
+
+    @property
+    def algorithmic_bytes(self) -> int:
+        """K and V read once, Q read and O written (bf16), LSE written (fp32)."""
+        qo = 2 * self.B * self.H * self.Nq * self.d * 2
+        return self.kv_bytes + qo + self.B * self.H * self.Nq * 4
+
+    def describe(self) -> str:
+        return (f"{self.name}: B={self.B} H={self.H} Nq={self.Nq} Nk={self.Nk} d={self.d} "
+                f"{'causal' if self.causal else 'non-causal'}")
+
+
+# Decode-shaped workload: one new token per sequence against a 32K context.
+DECODE_WORKLOAD = DecodeWorkload("decode_32k", 16, 32, 1, 32768, 128, False, 1240)
+
+
+def draw_decode_qkv(B: int, H: int, Nq: int, Nk: int, d: int, seed: int):
+    """Seeded bf16 q (B, H, Nq, d) and k, v (B, H, Nk, d), same recipe as draw_qkv."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn((B, H, Nq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
 def workload(index_or_name) -> Workload:
     for w in WORKLOADS:
         if w.index == index_or_name or w.name == index_or_name:

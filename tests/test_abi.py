@@ -128,3 +128,27 @@ def test_dynamic_argument_validation():
 def test_unit_count_limit():
     # B*H*ceil(N/256) beyond 2^30 is refused before any device work.
     assert fa.fa_fwd_raw(P, P, P, P, P, 1 << 12, 1 << 10, 1 << 17, 64, 0, 1.0, 0) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_decode_argument_validation_and_workspace_size():
+    W = 1 << 22
+    ok = (P, P, P, P, P, 2, 3, 1, 1000, 128, 0, 0.1, 0, W, 1 << 30, 0)
+    a = list(ok); a[13] = 0
+    assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_INVALID_ARG                 # NULL workspace
+    a = list(ok); a[7] = 17
+    assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_UNSUPPORTED                 # Nq > 16
+    a = list(ok); a[7] = 8; a[8] = 4; a[10] = 1
+    assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_INVALID_ARG                 # causal with Nq > Nk
+    a = list(ok); a[12] = 257
+    assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_INVALID_ARG                 # too many splits
+    a = list(ok); a[14] = 64
+    assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_INVALID_ARG                 # workspace too small
+    a = list(ok); a[13] = W + 16
+    assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_MISALIGNED                  # workspace alignment
+    a = list(ok); a[9] = 96
+    assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_UNSUPPORTED                 # d = 96
+    # workspace: splits x B*H x Nq x d fp32 partial outputs (256-byte padded) + partial LSEs
+    assert fa.decode_workspace_bytes(2, 3, 4, 1000, 128, 5) == 5 * 6 * 4 * 128 * 4 + 5 * 6 * 4 * 4
+    assert fa.decode_workspace_bytes(2, 3, 4, 1000, 128, 300) == 0
+    assert fa.decode_workspace_bytes(2, 3, 4, 1000, 128, 0) > 0
+    assert fa.fa_fwd_decode_raw(*ok) == fa.FA_ERR_NO_DEVICE                  # valid: stops at the device query

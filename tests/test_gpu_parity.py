@@ -349,3 +349,37 @@ def test_dynamic_full_size_and_strided(fa):
     o3, l3 = fa.fa_fwd(qb, kb, vb, causal=True, schedule="dynamic")
     torch.cuda.synchronize()
     assert torch.equal(o3, o1[:, :4]) and torch.equal(l3, l1[:, :4])
+
+
+# ---------------------------------------------------------------------------
+# Decode-shaped forward (fa_fwd_decode): few queries, long key sequences,
+# split over the keys and merged.
+# ---------------------------------------------------------------------------
+DECODE_CASES = [
+    (2, 4, 1, 4096, 128, False, 0), (2, 4, 1, 4097, 64, True, 0), (1, 8, 16, 3000, 128, True, 0),
+    (3, 2, 7, 130, 64, True, 3), (1, 2, 5, 5, 128, True, 0), (1, 1, 1, 1, 64, False, 0),
+    (2, 3, 3, 1000, 128, True, 1), (2, 3, 3, 1000, 128, False, 9), (1, 4, 12, 20000, 128, True, 0),
+]
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,d,causal,splits", DECODE_CASES)
+def test_decode_parity(fa, B, H, Nq, Nk, d, causal, splits):
+    q, k, v = synth.draw_decode_qkv(B, H, Nq, Nk, d, seed=300 + Nk + Nq)
+    qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
+    o, lse = fa.fa_fwd_decode(qd, kd, vd, causal=causal, num_splits=splits)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=causal, scale=1 / math.sqrt(d))
+    check(o, lse, O_ref, L_ref, f"decode B={B} H={H} Nq={Nq} Nk={Nk} d={d} causal={causal}")
+
+
+def test_decode_matches_square_last_rows(fa):
+    """Decode of the last Nq queries equals the last Nq rows of the square
+    causal problem computed by fa_fwd (within the parity tolerance)."""
+    B, H, N, d, Nq = 1, 4, 2000, 128, 8
+    q, k, v = synth.draw_qkv(B, H, N, d, seed=61)
+    qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
+    o_sq, l_sq = fa.fa_fwd(qd, kd, vd, causal=True)
+    o_dec, l_dec = fa.fa_fwd_decode(qd[:, :, N - Nq:].contiguous(), kd, vd, causal=True)
+    torch.cuda.synchronize()
+    assert float((o_dec.float() - o_sq[:, :, N - Nq:].float()).abs().max()) <= TOL_MAX
+    assert float((l_dec - l_sq[:, :, N - Nq:]).abs().max()) <= TOL_LSE
