@@ -14,6 +14,8 @@ online softmax by hand".
 from .exact_attention import (  # noqa: F401
     bf16_bits_to_f64,
     attention_fp64,
+    attention_bwd_fp64,
+    attention_bwd_rows_fp64,
     attention_rows_fp64,
     softmax_rows_fp64,
     online_softmax_row_blockmax,

@@ -29,6 +29,10 @@ first page's "The Tiling Strategy" pseudocode.  They exist only so the
 self-tests can check that tiling reaches the direct result; the oracle proper
 is the direct (materialising) definition.
 
+The backward functions differentiate that definition (formulas in the
+backward section below); the page's backward paragraph (same section as the
+saved statistic) only says P is recomputed from Q, K, V and the statistics.
+
 Parity is pinned by the CPU tests (worked example, exercise 1, closed forms,
 invariants, brute force and an independent library routine); nothing here is
 "parity unpinned".
@@ -150,6 +154,102 @@ def attention_fp64(q, k, v, causal: bool = False, scale: float | None = None,
                 O[b, h, r0:r1], LSE[b, h, r0:r1] = attention_rows_fp64(
                     q[b, h], k[b, h], v[b, h], rows, causal, scale, key_offset)
     return O, LSE
+
+
+# ---------------------------------------------------------------------------
+# Backward pass (gradients of the direct definition)
+# ---------------------------------------------------------------------------
+#
+# The page "Flash attention optimization", section "Sizing a tile, and why the
+# backward pass recomputes instead of storing", says the backward pass needs P
+# again and rebuilds it from the saved Q, K, V and per-row statistics instead
+# of storing it; it prints no gradient formula.  The oracle therefore
+# differentiates the forward definition above.  For a scalar loss with upstream
+# gradient dO = dL/dO, and with S = scale * Q K^T (masked), P = softmax(S)
+# row-wise, O = P V:
+#
+#   dV = P^T dO                       (O is linear in V)
+#   dP = dO V^T
+#   D_i = sum_t dO_it O_it            (= sum_j P_ij dP_ij)
+#   dS = P * (dP - D[:, None])        (Jacobian of the row softmax)
+#   dQ = scale * dS K,   dK = scale * dS^T Q
+#
+# P is recomputed exactly as in the forward (global-max subtraction), so masked
+# entries are exactly 0 and contribute nothing.
+
+def attention_bwd_rows_fp64(q_bh, k_bh, v_bh, do_bh, rows, causal: bool, scale: float,
+                            key_offset: int = 0):
+    """Gradient contributions of selected query rows of one (batch, head).
+
+    q_bh, do_bh: (N_q, d); k_bh, v_bh: (N_k, d) float64.  Materialises
+    S[rows, :] and P[rows, :] over all keys, then applies the formulas above.
+    Returns (dQ_rows (len(rows), d), dK_part (N_k, d), dV_part (N_k, d),
+    D_rows (len(rows),)): dQ of these rows is complete; dK and dV are the sums
+    over these rows only (the caller adds the parts of all row chunks).  Rows
+    with no allowed key (causal, N_q > N_k) contribute nothing.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    N = k_bh.shape[0]
+    S = scale * (q_bh[rows] @ k_bh.T)                       # S = Q K^T * scale
+    if causal:
+        allowed = np.arange(N, dtype=np.int64)[None, :] <= rows[:, None] + key_offset
+        S = np.where(allowed, S, -np.inf)
+        keep = allowed.any(axis=1)
+        if not keep.all():
+            dQ = np.zeros((len(rows), q_bh.shape[1]))
+            D = np.zeros(len(rows))
+            dK = np.zeros_like(k_bh)
+            dV = np.zeros_like(v_bh)
+            if keep.any():
+                dQ[keep], dK, dV, D[keep] = attention_bwd_rows_fp64(
+                    q_bh, k_bh, v_bh, do_bh, rows[keep], causal, scale, key_offset)
+            return dQ, dK, dV, D
+    P, _, _ = softmax_rows_fp64(S)                          # P recomputed
+    dO = do_bh[rows]
+    O = P @ v_bh                                            # O = P V
+    dV = P.T @ dO                                           # dV = P^T dO
+    dP = dO @ v_bh.T                                        # dP = dO V^T
+    D = np.sum(dO * O, axis=1)                              # D_i = dO_i . O_i
+    dS = P * (dP - D[:, None])                              # softmax Jacobian
+    dQ = scale * (dS @ k_bh)                                # dQ = scale dS K
+    dK = scale * (dS.T @ q_bh[rows])                        # dK = scale dS^T Q
+    return dQ, dK, dV, D
+
+
+def attention_bwd_fp64(q, k, v, do, causal: bool = False, scale: float | None = None,
+                       row_chunk: int = 512):
+    """Exact attention backward in float64: q, do (B, H, N_q, d); k, v (B, H, N_k, d).
+
+    Returns (dQ, dK, dV, D) as float64 arrays of the inputs' shapes (D has
+    shape (B, H, N_q)).  Rows are processed ``row_chunk`` at a time; dK and dV
+    are the sums of the chunks' parts.  Causal masking follows the forward:
+    query i may see key j iff j <= i + N_k - N_q.
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    if q.ndim != 4 or k.ndim != 4 or v.shape != k.shape or q.shape[:2] != k.shape[:2] \
+            or q.shape[3] != k.shape[3] or do.shape != q.shape:
+        raise ValueError("q and do must be (B, H, N_q, d) and k, v (B, H, N_k, d)")
+    B, H, N, d = q.shape
+    key_offset = k.shape[2] - N
+    if causal and key_offset < 0:
+        raise ValueError("causal attention needs N_q <= N_k")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = np.empty_like(q)
+    dK = np.zeros_like(k)
+    dV = np.zeros_like(v)
+    D = np.empty((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, N, row_chunk):
+                rows = np.arange(r0, min(N, r0 + row_chunk))
+                dq, dk, dv, dd = attention_bwd_rows_fp64(q[b, h], k[b, h], v[b, h], do[b, h],
+                                                         rows, causal, scale, key_offset)
+                dQ[b, h, rows] = dq
+                dK[b, h] += dk
+                dV[b, h] += dv
+                D[b, h, rows] = dd
+    return dQ, dK, dV, D
 
 
 # ---------------------------------------------------------------------------
