@@ -488,6 +488,66 @@ def run_decode(args):
     return 0
 
 
+def run_bwd(args):
+    """Backward pass of the headline workload: one step = fa_bwd (D pre-pass,
+    the main gradient kernel, dQ conversion) on inputs and forward outputs
+    already in device memory.  FLOPs: the five matrix products of the
+    recomputing backward (S, dP, dV, dK, dQ), 2.5x the forward's count."""
+    import torch
+
+    import exact_attention_122_b200 as fa
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = synth.workload(args.workload)
+    q, k, v = (t.to(dev) for t in synth.workload_qkv(w))
+    dout = synth.draw_dout(w.B, w.H, w.N, w.d, seed=w.seed).to(dev)
+    stream = torch.cuda.Stream(device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.bwd_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        fa.fa_fwd(q, k, v, causal=w.causal, out=o, lse=lse, stream=stream)
+
+    def step():
+        fa.fa_bwd(q, k, v, o, lse, dout, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws,
+                  stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+    st, word = fa.device_status(stream.cuda_stream)
+    if st != fa.FA_OK:
+        raise SystemExit(f"kernel status {fa.status_string(st)} {word:#x}")
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 2.5 * w.flops
+    value = flops / (ms / 1e3) / 1e12
+    peak, peak_sus, peak_src = load_peaks()
+    line = {"metric": "attention backward TFLOP/s (1 GPU)", "value": value, "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "causal": w.causal, "flops_per_step": flops,
+                       "l2": "inputs 537 MB > 126 MB L2; no flush"},
+            "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s",
+                         "frac": value / peak, "traffic": None, "peak_source": peak_src,
+                         "kernel": "bwd_prep + bwd_kernel + bwd_dq_out (whole step)"},
+            "gpu_launches": 3 * args.steps, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_sweep(args):
     import torch
 
@@ -548,6 +608,8 @@ def main(argv=None):
                          "on the long causal workloads) or fa_fwd (static)")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode-shaped path (HBM-bound) instead of the headline line")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward pass (fa_bwd) of the workload instead of the forward")
     ap.add_argument("--sweep", action="store_true",
                     help="print the sequence-length sweep curve instead of the headline line")
     args = ap.parse_args(argv)
@@ -557,6 +619,8 @@ def main(argv=None):
         raise SystemExit("--steps must be >= 1")
     if args.sweep:
         return run_sweep(args)
+    if args.bwd:
+        return run_bwd(args)
     if args.decode:
         return run_decode(args)
     w = synth.workload(args.workload)

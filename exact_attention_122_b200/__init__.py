@@ -1,4 +1,4 @@
-"""exact_attention_122_b200 -- exact attention forward on B200 (sm_100a).
+"""exact_attention_122_b200 -- exact attention forward and backward on B200 (sm_100a).
 
 The computation lives in the CUDA library libfa_b200.so behind the C ABI of
 include/fa.h; this module only marshals arguments to it (torch supplies
@@ -12,5 +12,5 @@ from ._binding import (  # noqa: F401
     DECODE_MAX_QUERIES, DECODE_MAX_SPLITS, decode_workspace_bytes, fa_fwd_decode, fa_fwd_decode_raw,
     FaError, library, library_path, status_string, version,
     fa_fwd, fa_fwd_raw, fa_fwd_strided_raw, fa_fwd_dynamic_raw, fa_fwd_dynamic_noalloc_raw,
-    fa_fwd_debug_raw, device_status,
+    fa_fwd_debug_raw, device_status, bwd_workspace_bytes, fa_bwd, fa_bwd_raw,
 )

@@ -15,7 +15,8 @@ FA_ERR_TIMEOUT = 5
 FA_ERR_NO_DEVICE = 6
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_dynamic_noalloc",
-                    "fa_fwd_decode_workspace_bytes", "fa_fwd_decode", "fa_fwd_debug",
+                    "fa_fwd_decode_workspace_bytes", "fa_fwd_decode", "fa_bwd_workspace_bytes",
+                    "fa_bwd", "fa_fwd_debug",
                     "fa_get_device_status", "fa_status_string", "fa_last_cuda_error", "fa_version")
 DECODE_MAX_QUERIES = 16                # FA_DECODE_MAX_QUERIES
 DECODE_MAX_SPLITS = 256                # FA_DECODE_MAX_SPLITS
@@ -56,6 +57,11 @@ def library() -> ctypes.CDLL:
     lib.fa_fwd_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.fa_fwd_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, ctypes.c_size_t, vp]
     lib.fa_fwd_decode.restype = i
+    lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
+    lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp,
+                           ctypes.c_size_t, vp]
+    lib.fa_bwd.restype = i
     lib.fa_fwd_debug.argtypes = fwd_args + [u, i]
     lib.fa_fwd_debug.restype = i
     lib.fa_get_device_status.argtypes = [vp, ctypes.POINTER(u)]
@@ -170,6 +176,55 @@ def fa_fwd_decode(q, k, v, causal: bool = False, scale: float | None = None, num
     if st != FA_OK:
         raise FaError(st, "fa_fwd_decode")
     return out, lse
+
+
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(library().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def fa_bwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr: int,
+               dq_ptr: int, dk_ptr: int, dv_ptr: int, B: int, H: int, N: int, d: int, causal: int,
+               scale: float, ws_ptr: int, ws_bytes: int, stream_ptr: int) -> int:
+    """Direct call of fa_bwd; returns the fa_status code."""
+    return library().fa_bwd(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr,
+                            B, H, N, d, causal, scale, ws_ptr, ws_bytes, stream_ptr)
+
+
+def fa_bwd(q, k, v, out, lse, dout, causal: bool = False, scale: float | None = None,
+           dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of attention for contiguous bf16 CUDA tensors q, k, v, out,
+    dout (B, H, N, d) and the forward's fp32 lse (B, H, N).  ``workspace`` (at
+    least bwd_workspace_bytes(B, H, N, d) bytes of device memory) is allocated
+    with torch when not given."""
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    B, H, N, d = q.shape
+    for t in (k, v, out, dout):
+        if t.shape != q.shape:
+            raise ValueError("q, k, v, out and dout must have one shape (B, H, N, d)")
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.shape == (B, H, N)
+            and lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor (B, H, N)")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        st = fa_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                        lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                        1 if causal else 0, float(scale), workspace.data_ptr(),
+                        workspace.numel() * workspace.element_size(), s.cuda_stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd")
+    return dq, dk, dv
 
 
 _WORKSPACES = {}

@@ -1,0 +1,801 @@
+// fa_bwd_sm100.cu -- exact attention backward for B200 (sm_100a).
+//
+// Given Q, K, V, the forward's output O and per-row log-sum-exp LSE, and the
+// upstream gradient dO, computes dQ, dK, dV of O = softmax(scale Q K^T
+// [+ causal mask]) V without storing P: every P block is rebuilt from Q, K
+// and LSE on chip (page "Flash attention optimization", section "Sizing a
+// tile, and why the backward pass recomputes instead of storing": only the
+// per-row statistics are kept and the needed P blocks are recomputed from the
+// saved Q, K, V tiles).  The gradient formulas are those of the softmax:
+//   P = exp(scale S - LSE),  dV = P^T dO,  dP = dO V^T,
+//   D_i = sum_t dO_it O_it,  dS = P * (dP - D),
+//   dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels, all on the caller's stream:
+//   bwd_prep     D_i and LSE_i * log2(e) per row into the workspace (padded
+//                rows get D = 0, LSE = +inf, so their P is 0), and zeroes
+//                the fp32 dQ accumulator.
+//   bwd_kernel   one CTA per 128-key block of one (batch, head), 448 threads:
+//                  warps 0-7   compute: P, dS for the key block's 128 rows
+//                              (warp w: TMEM lane quarter w % 4, half of the
+//                              query columns w / 4)
+//                  warps 8-11  dQ drain: read this step's dQ partial from
+//                              TMEM and add it to the fp32 accumulator in
+//                              global memory with coalesced reductions
+//                  warp  12    MMA issuer (one thread)
+//                  warp  13    TMA producer (one thread): K, V once, then
+//                              Q, dO, LSE, D of each query block through an
+//                              NS-stage ring
+//                K_j, V_j stay in shared memory and dK_j, dV_j accumulate in
+//                TMEM over all query blocks; per query block of BQ rows the
+//                tensor core computes S^T = K Q^T and dP^T = V dO^T (keys on
+//                the TMEM lanes), then dV += P^T dO (P from TMEM), dK += dS^T Q
+//                and the dQ partial (dS from shared memory).  The MMAs of
+//                block i-1's gradients are issued after block i's S^T and
+//                dP^T, so the compute warps' exponentials for block i overlap
+//                the tensor core's work on block i-1.
+//   bwd_dq_out   dQ = bf16(scale * accumulator).
+//
+// Every mbarrier wait is bounded by a %globaltimer watchdog, as in the
+// forward kernel: a wait that runs out records FA_ERR_TIMEOUT in
+// g_bwd_status, raises a CTA-wide abort flag, and every role leaves its
+// loop, drains its own copies and MMAs (bounded), frees TMEM and returns.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "fa.h"
+#include "fa_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace bwd {
+
+using namespace sm100;
+
+constexpr int BK = 128;             // keys per CTA (TMEM lanes of S^T, dP^T, dK, dV)
+constexpr int NUM_THREADS = 448;
+constexpr int COMPUTE_WARPS = 8;
+constexpr int DQ_WARP0 = 8;
+constexpr int MMA_WARP = 12;
+constexpr int TMA_WARP = 13;
+constexpr int NS = 2;               // Q / dO ring stages
+constexpr float LOG2E = 1.4426950408889634f;
+
+enum : uint32_t { ROLE_COMPUTE = 1u, ROLE_MMA = 2u, ROLE_PRODUCER = 3u, ROLE_DQ = 4u,
+                  ROLE_DRAIN = 5u };
+
+// D = 128: 64 query rows per step and dQ^T (d on the TMEM lanes, M = 128).
+// D = 64:  128 query rows per step and dQ (queries on the lanes, M = 128).
+// Both keep every MMA at M = 128 and fit the 512 TMEM columns.
+template <int D>
+struct Cfg {
+    static constexpr int BQ = D == 128 ? 64 : 128;
+    static constexpr bool DQ_T = D == 128;
+    static constexpr int NP = D == 128 ? 2 : 1;         // P buffers in TMEM
+    static constexpr int KV_BYTES = BK * D * 2;
+    static constexpr int KV_SLAB = BK * 128;             // 64 columns of a K/V tile
+    static constexpr int QD_BYTES = BQ * D * 2;
+    static constexpr int QD_SLAB = BQ * 128;             // 64 columns of a Q/dO tile
+    static constexpr int DS_BYTES = BK * BQ * 2;
+    static constexpr int DS_SLAB = BK * 128;             // 64 queries of dS, all keys
+    static constexpr int VEC_BYTES = 2 * BQ * 4;         // LSE2 and D of one query block
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + KV_BYTES;
+    static constexpr int OFF_Q = OFF_V + KV_BYTES;
+    static constexpr int OFF_DO = OFF_Q + NS * QD_BYTES;
+    static constexpr int OFF_DS = OFF_DO + NS * QD_BYTES;
+    static constexpr int OFF_VEC = OFF_DS + 2 * DS_BYTES;
+    static constexpr int OFF_BAR = OFF_VEC + NS * VEC_BYTES;
+    static constexpr int B_KV_FULL = 0;
+    static constexpr int B_QD_FULL = 1;                  // [NS]
+    static constexpr int B_QD_EMPTY = 1 + NS;            // [NS]
+    static constexpr int B_SDP_FULL = 1 + 2 * NS;
+    static constexpr int B_SDP_FREE = 2 + 2 * NS;
+    static constexpr int B_DS_READY = 3 + 2 * NS;        // [2]
+    static constexpr int B_P_FREE = 5 + 2 * NS;          // [2]
+    static constexpr int B_DS_FREE = 7 + 2 * NS;         // [2]
+    static constexpr int B_DQ_FULL = 9 + 2 * NS;
+    static constexpr int B_DQ_EMPTY = 10 + 2 * NS;
+    static constexpr int B_ACC_FULL = 11 + 2 * NS;
+    static constexpr int B_DRAIN = 12 + 2 * NS;
+    static constexpr int NUM_BARS = 13 + 2 * NS;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem base, abort flag
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+    // TMEM columns
+    static constexpr uint32_t TM_S = 0;
+    static constexpr uint32_t TM_DP = BQ;
+    static constexpr uint32_t TM_P = 2 * BQ;                   // NP buffers of BQ/2 columns
+    static constexpr uint32_t TM_DQ = TM_P + NP * (BQ / 2);    // dQ^T: BQ cols; dQ: D cols
+    static constexpr uint32_t DQ_COLS = DQ_T ? BQ : D;
+    static constexpr uint32_t TM_DV = TM_DQ + DQ_COLS;
+    static constexpr uint32_t TM_DK = TM_DV + D;
+    static constexpr uint32_t TM_COLS = 512;
+    static_assert(TM_DK + D <= TM_COLS, "TMEM budget");
+    static_assert(ALLOC <= 227 * 1024, "shared memory budget");
+    static_assert(BYTES > 116 * 1024, "one CTA per SM keeps TMEM allocation uncontended");
+    static_assert((BQ / 2) % 32 == 0, "compute warps take 32-column chunks");
+};
+
+__device__ unsigned int g_bwd_status;   // 0 = fine; else (FA_ERR_TIMEOUT << 24) | role << 20 | block
+
+struct Watchdog {
+    volatile int* abort_flag;
+    uint64_t limit_ns;
+};
+
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Watchdog wd,
+                                           uint32_t role, uint32_t blk) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*wd.abort_flag) return false;
+        if (global_timer_ns() - t0 > wd.limit_ns) {
+            atomicCAS(&g_bwd_status, 0u,
+                      (uint32_t(FA_ERR_TIMEOUT) << 24) | (role << 20) | (blk & 0xFFFFFu));
+            *wd.abort_flag = 1;
+            __threadfence_block();
+            return false;
+        }
+    }
+}
+
+// wait_phase taken by a whole warp: the warp goes on only if every lane's
+// wait succeeded, so the warp-collective tcgen05 loads and stores that follow
+// are never reached by part of a warp.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, Watchdog wd,
+                                          uint32_t role, uint32_t blk) {
+    const bool ok = wait_phase(bar, parity, wd, role, blk);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait that ignores the abort flag: used only to drain this thread's
+// own copies and MMAs before the CTA exits.
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns) {
+            atomicCAS(&g_bwd_status, 0u, (uint32_t(FA_ERR_TIMEOUT) << 24) | (ROLE_DRAIN << 20));
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ void cta_sync() {
+    asm volatile("bar.sync 0, %0;" ::"n"(NUM_THREADS) : "memory");
+}
+
+// 1-D bulk copy global -> shared completing on an mbarrier (16-byte aligned
+// addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Pre-pass: D_i = dO_i . O_i (fp32), LSE2_i = LSE_i log2(e), zero dQ_acc.
+// Rows r in [N, Npad) get D = 0 and LSE2 = +inf.  D / 8 threads per row, each
+// on 8 consecutive elements.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict__ o,
+                                                const __nv_bfloat16* __restrict__ dout,
+                                                const float* __restrict__ lse,
+                                                float* __restrict__ lse2, float* __restrict__ dvec,
+                                                float* __restrict__ dq_acc, long long BH, int N,
+                                                int Npad) {
+    constexpr int TPR = D / 8;                          // threads per row
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long row = t / TPR;                      // over BH * Npad
+    const int part = int(t % TPR);
+    const bool live = row < BH * Npad;                  // every lane joins the shuffles below
+    const long long bh = row / Npad;
+    const int r = int(row - bh * Npad);
+    float acc = 0.f;
+    if (live && r < N) {
+        const long long e = ((bh * N + r) * D) + part * 8;
+        const uint4 a = *reinterpret_cast<const uint4*>(o + e);
+        const uint4 b = *reinterpret_cast<const uint4*>(dout + e);
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 x = __bfloat1622float2(a2[i]);
+            const float2 y = __bfloat1622float2(b2[i]);
+            acc = fmaf(x.x, y.x, acc);
+            acc = fmaf(x.y, y.y, acc);
+        }
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (!live) return;
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (part == 0) {
+        dvec[row] = r < N ? acc : 0.f;
+        lse2[row] = r < N ? lse[bh * N + r] * LOG2E : INFINITY;
+    }
+}
+
+// dQ = bf16(scale * dQ_acc) for rows < N; 8 elements per thread.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_out(const float* __restrict__ dq_acc,
+                                                  __nv_bfloat16* __restrict__ dq, long long BH,
+                                                  int N, int Npad, float scale) {
+    constexpr int TPR = D / 8;
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long row = t / TPR;                      // over BH * N
+    const int part = int(t % TPR);
+    if (row >= BH * N) return;
+    const long long bh = row / N;
+    const long long r = row - bh * N;
+    const float4* a = reinterpret_cast<const float4*>(dq_acc + (bh * Npad + r) * D + part * 8);
+    const float4 x = a[0], y = a[1];
+    uint4 out;
+    out.x = pack_bf16x2(scale * x.x, scale * x.y);
+    out.y = pack_bf16x2(scale * x.z, scale * x.w);
+    out.z = pack_bf16x2(scale * y.x, scale * y.y);
+    out.w = pack_bf16x2(scale * y.z, scale * y.w);
+    *reinterpret_cast<uint4*>(dq + row * D + part * 8) = out;
+}
+
+// ---------------------------------------------------------------------------
+// Main kernel
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+           const float* __restrict__ lse2, const float* __restrict__ dvec,
+           float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
+           __nv_bfloat16* __restrict__ dv, int BH, int H, int N, int Npad, int causal,
+           float scale, unsigned long long watchdog_ns) {
+    using C = Cfg<D>;
+    constexpr int BQ = C::BQ;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+
+    // Work: key-block-major order, so every head's longest causal blocks
+    // (the first key blocks) are scheduled first.
+    const int nkb = (N + BK - 1) / BK;
+    const int kb = int(blockIdx.x / unsigned(BH));
+    const int bh = int(blockIdx.x - unsigned(kb) * unsigned(BH));
+    const int b = bh / H, h = bh - (bh / H) * H;
+    const int k0 = kb * BK;
+    const int nqb = (N + BQ - 1) / BQ;
+    const int qb_first = causal ? k0 / BQ : 0;
+    const int nsteps = nqb - qb_first;
+    (void)nkb;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::B_KV_FULL), 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(C::B_QD_FULL + s), 1);
+            mbar_init(bar(C::B_QD_EMPTY + s), 1 + COMPUTE_WARPS);
+        }
+        mbar_init(bar(C::B_SDP_FULL), 1);
+        mbar_init(bar(C::B_SDP_FREE), COMPUTE_WARPS);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(C::B_DS_READY + i), COMPUTE_WARPS);
+            mbar_init(bar(C::B_P_FREE + i), 1);
+            mbar_init(bar(C::B_DS_FREE + i), 1);
+        }
+        mbar_init(bar(C::B_DQ_FULL), 1);
+        mbar_init(bar(C::B_DQ_EMPTY), 4);
+        mbar_init(bar(C::B_ACC_FULL), 1);
+        mbar_init(bar(C::B_DRAIN), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), C::TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    cta_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Watchdog wd{abort_flag, watchdog_ns};
+    const uint32_t blk_id = blockIdx.x;
+
+    if (warp == TMA_WARP) {
+        // ------------------------------------------------------------------
+        // Producer
+        // ------------------------------------------------------------------
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar(C::B_KV_FULL), 2 * C::KV_BYTES);
+#pragma unroll
+            for (int sl = 0; sl < D / 64; ++sl) {
+                tma_load_4d(sbase + C::OFF_K + sl * C::KV_SLAB, &tmK, sl * 64, k0, h, b,
+                            bar(C::B_KV_FULL));
+                tma_load_4d(sbase + C::OFF_V + sl * C::KV_SLAB, &tmV, sl * 64, k0, h, b,
+                            bar(C::B_KV_FULL));
+            }
+            int issued = 0;
+            for (int n = 0; n < nsteps; ++n) {
+                const int s = n % NS;
+                if (n >= NS && !wait_phase(bar(C::B_QD_EMPTY + s), ((n / NS) - 1) & 1, wd,
+                                           ROLE_PRODUCER, blk_id))
+                    break;
+                const int q0 = (qb_first + n) * BQ;
+                const uint32_t full = bar(C::B_QD_FULL + s);
+                mbar_arrive_expect_tx(full, 2 * C::QD_BYTES + C::VEC_BYTES);
+#pragma unroll
+                for (int sl = 0; sl < D / 64; ++sl) {
+                    tma_load_4d(sbase + C::OFF_Q + s * C::QD_BYTES + sl * C::QD_SLAB, &tmQ,
+                                sl * 64, q0, h, b, full);
+                    tma_load_4d(sbase + C::OFF_DO + s * C::QD_BYTES + sl * C::QD_SLAB, &tmDO,
+                                sl * 64, q0, h, b, full);
+                }
+                const long long vrow = (long long)bh * Npad + q0;
+                bulk_load(sbase + C::OFF_VEC + s * C::VEC_BYTES, lse2 + vrow, BQ * 4, full);
+                bulk_load(sbase + C::OFF_VEC + s * C::VEC_BYTES + BQ * 4, dvec + vrow, BQ * 4,
+                          full);
+                ++issued;
+            }
+            // Drain: every copy this thread issued has landed before exit.
+            wait_drain(bar(C::B_KV_FULL), 0, watchdog_ns);
+            for (int n = (issued > NS ? issued - NS : 0); n < issued; ++n)
+                wait_drain(bar(C::B_QD_FULL + n % NS), (n / NS) & 1, watchdog_ns);
+        }
+    } else if (warp == MMA_WARP) {
+        // ------------------------------------------------------------------
+        // MMA issuer
+        // ------------------------------------------------------------------
+        if (lane == 0) {
+            constexpr uint32_t ID_S = idesc_bf16(128, BQ, false);          // S^T, dP^T
+            constexpr uint32_t ID_G = idesc_bf16(128, D, true);            // dV, dK
+            constexpr uint32_t ID_Q = C::DQ_T ? idesc_bf16(128, BQ, true, true)   // dQ^T
+                                              : idesc_bf16(128, D, true, true);   // dQ
+            const uint64_t dK_kmaj = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
+            const uint64_t dV_kmaj = sdesc_sw128(sbase + C::OFF_V, 16, 1024);
+            const uint64_t dK_mn = sdesc_sw128(sbase + C::OFF_K, C::KV_SLAB, 1024);
+            bool ok = wait_phase(bar(C::B_KV_FULL), 0, wd, ROLE_MMA, blk_id);
+            tc_fence_after();
+
+            auto grads = [&](int m) -> bool {
+                const int s = m % NS, pb = m % C::NP, db = m % 2;
+                if (!wait_phase(bar(C::B_DS_READY + db), (m / 2) & 1, wd, ROLE_MMA, blk_id))
+                    return false;
+                tc_fence_after();
+                const uint32_t sq = sbase + C::OFF_Q + s * C::QD_BYTES;
+                const uint32_t sdo = sbase + C::OFF_DO + s * C::QD_BYTES;
+                const uint32_t sds = sbase + C::OFF_DS + db * C::DS_BYTES;
+                // dV += P^T dO: A = P (TMEM, 16 queries = 8 columns per step),
+                // B = dO MN-major (16 query rows of 128 bytes per step).
+                const uint64_t do_mn = sdesc_sw128(sdo, C::QD_SLAB, 1024);
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    mma_ts(tmem + C::TM_DV, tmem + C::TM_P + pb * (BQ / 2) + kk * 8,
+                           desc_add(do_mn, uint32_t((kk * 2048) >> 4)), ID_G,
+                           (m > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(bar(C::B_P_FREE + pb));
+                // dK += dS^T Q: A = dS K-major (keys x queries), B = Q MN-major.
+                const uint64_t ds_kmaj = sdesc_sw128(sds, 16, 1024);
+                const uint64_t q_mn = sdesc_sw128(sq, C::QD_SLAB, 1024);
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    mma_ss(tmem + C::TM_DK,
+                           desc_add(ds_kmaj, uint32_t(((kk / 4) * C::DS_SLAB + (kk % 4) * 32) >> 4)),
+                           desc_add(q_mn, uint32_t((kk * 2048) >> 4)), ID_G,
+                           (m > 0 || kk > 0) ? 1u : 0u);
+                // dQ partial of this query block: K = 128 keys in steps of 16.
+                if (m >= 1 && !wait_phase(bar(C::B_DQ_EMPTY), (m - 1) & 1, wd, ROLE_MMA, blk_id))
+                    return false;
+                tc_fence_after();
+                const uint64_t ds_mn = sdesc_sw128(sds, C::DS_SLAB, 1024);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t off = uint32_t((kk * 2048) >> 4);
+                    if (C::DQ_T)   // dQ^T = K^T dS^T: A = K MN-major (d x keys), B = dS^T MN-major
+                        mma_ss(tmem + C::TM_DQ, desc_add(dK_mn, off), desc_add(ds_mn, off), ID_Q,
+                               kk > 0 ? 1u : 0u);
+                    else           // dQ = dS K: A = dS MN-major (queries x keys), B = K MN-major
+                        mma_ss(tmem + C::TM_DQ, desc_add(ds_mn, off), desc_add(dK_mn, off), ID_Q,
+                               kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(C::B_DQ_FULL));
+                tc_commit(bar(C::B_DS_FREE + db));
+                tc_commit(bar(C::B_QD_EMPTY + s));
+                return true;
+            };
+
+            for (int n = 0; ok && n < nsteps; ++n) {
+                const int s = n % NS;
+                if (!wait_phase(bar(C::B_QD_FULL + s), (n / NS) & 1, wd, ROLE_MMA, blk_id)) {
+                    ok = false;
+                    break;
+                }
+                if (n >= 1 && !wait_phase(bar(C::B_SDP_FREE), (n - 1) & 1, wd, ROLE_MMA, blk_id)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sq = sbase + C::OFF_Q + s * C::QD_BYTES;
+                const uint32_t sdo = sbase + C::OFF_DO + s * C::QD_BYTES;
+                const uint64_t q_kmaj = sdesc_sw128(sq, 16, 1024);
+                const uint64_t do_kmaj = sdesc_sw128(sdo, 16, 1024);
+                // S^T = K Q^T and dP^T = V dO^T: M = 128 keys, N = BQ queries, K = d.
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t oa = uint32_t(((kk / 4) * C::KV_SLAB + (kk % 4) * 32) >> 4);
+                    const uint32_t ob = uint32_t(((kk / 4) * C::QD_SLAB + (kk % 4) * 32) >> 4);
+                    mma_ss(tmem + C::TM_S, desc_add(dK_kmaj, oa), desc_add(q_kmaj, ob), ID_S,
+                           kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t oa = uint32_t(((kk / 4) * C::KV_SLAB + (kk % 4) * 32) >> 4);
+                    const uint32_t ob = uint32_t(((kk / 4) * C::QD_SLAB + (kk % 4) * 32) >> 4);
+                    mma_ss(tmem + C::TM_DP, desc_add(dV_kmaj, oa), desc_add(do_kmaj, ob), ID_S,
+                           kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(C::B_SDP_FULL));
+                if (n >= 1 && !grads(n - 1)) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (ok) ok = grads(nsteps - 1);
+            if (ok) tc_commit(bar(C::B_ACC_FULL));
+            // Drain: every MMA this thread issued has completed before TMEM is freed.
+            tc_commit(bar(C::B_DRAIN));
+            wait_drain(bar(C::B_DRAIN), 0, watchdog_ns);
+        }
+    } else if (warp >= DQ_WARP0) {
+        // ------------------------------------------------------------------
+        // dQ drain: TMEM -> fp32 reductions into dq_acc
+        // ------------------------------------------------------------------
+        const int qw = warp - DQ_WARP0;                       // lane quarter
+        const uint32_t lane_base = uint32_t(32 * qw) << 16;
+        for (int n = 0; n < nsteps; ++n) {
+            if (!warp_wait(bar(C::B_DQ_FULL), n & 1, wd, ROLE_DQ, blk_id)) break;
+            tc_fence_after();
+            const int q0 = (qb_first + n) * BQ;
+            if (C::DQ_T) {
+                // lane = d index t; columns = the BQ queries of the block
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_base + C::TM_DQ, r0);
+                tmem_ld32(tmem + lane_base + C::TM_DQ + 32, r1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
+                const int t = 32 * qw + lane;
+                float* base = dq_acc + ((long long)bh * Npad + q0) * D + t;
+                const int rows = min(BQ, N - q0);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (j < rows) red_add_f32(base + (long long)j * D, __uint_as_float(r0[j]));
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (32 + j < rows)
+                        red_add_f32(base + (long long)(32 + j) * D, __uint_as_float(r1[j]));
+            } else {
+                // lane = query row; columns = d
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_base + C::TM_DQ, r0);
+                tmem_ld32(tmem + lane_base + C::TM_DQ + 32, r1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
+                const int row = q0 + 32 * qw + lane;
+                if (row < N) {
+                    float* base = dq_acc + ((long long)bh * Npad + row) * D;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        red_add_v4_f32(base + j, __uint_as_float(r0[j]), __uint_as_float(r0[j + 1]),
+                                       __uint_as_float(r0[j + 2]), __uint_as_float(r0[j + 3]));
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        red_add_v4_f32(base + 32 + j, __uint_as_float(r1[j]),
+                                       __uint_as_float(r1[j + 1]), __uint_as_float(r1[j + 2]),
+                                       __uint_as_float(r1[j + 3]));
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------
+        // Compute warps: P and dS for key rows r (TMEM lane), half of the
+        // query columns each.
+        // ------------------------------------------------------------------
+        const int qw = warp % 4, half = warp / 4;
+        const int r = 32 * qw + lane;                         // key row in the block
+        const int key = k0 + r;
+        const uint32_t lane_base = uint32_t(32 * qw) << 16;
+        const float cs = scale * LOG2E;
+        bool ok = true;
+        for (int n = 0; ok && n < nsteps; ++n) {
+            const int s = n % NS, pb = n % C::NP, db = n % 2;
+            const int q0 = (qb_first + n) * BQ;
+            // QD_FULL: the LSE2 / D vectors of this block (bulk copies) have
+            // landed; SDP_FULL: S^T and dP^T are in TMEM.
+            if (!warp_wait(bar(C::B_QD_FULL + s), (n / NS) & 1, wd, ROLE_COMPUTE, blk_id) ||
+                !warp_wait(bar(C::B_SDP_FULL), n & 1, wd, ROLE_COMPUTE, blk_id)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const bool need_mask = (causal && q0 < k0 + BK) || (q0 + BQ > N) || (k0 + BK > N);
+            const float* vl = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * C::VEC_BYTES);
+            const float* vd = vl + BQ;
+            const uint32_t sds = sbase + C::OFF_DS + db * C::DS_BYTES;
+            constexpr int CHUNKS = (BQ / 2) / 32;
+#pragma unroll 1
+            for (int c = 0; c < CHUNKS; ++c) {
+                const int col0 = half * (BQ / 2) + c * 32;
+                uint32_t sv[32], dpv[32];
+                tmem_ld32(tmem + lane_base + C::TM_S + col0, sv);
+                tmem_ld32(tmem + lane_base + C::TM_DP + col0, dpv);
+                if (c == CHUNKS - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(C::B_SDP_FREE));
+                }
+                uint32_t pu[16], du[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(vl + col0 + j);
+                    const float4 d4 = *reinterpret_cast<const float4*>(vd + col0 + j);
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float p[4], ds[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        p[u] = ex2(fmaf(__uint_as_float(sv[j + u]), cs, -lv[u]));
+                        if (need_mask) {
+                            const int qi = q0 + col0 + j + u;
+                            if ((causal && qi < key) || qi >= N || key >= N) p[u] = 0.f;
+                        }
+                        ds[u] = p[u] * (__uint_as_float(dpv[j + u]) - dd[u]);
+                    }
+                    pu[j / 2] = pack_bf16x2(p[0], p[1]);
+                    pu[j / 2 + 1] = pack_bf16x2(p[2], p[3]);
+                    du[j / 2] = pack_bf16x2(ds[0], ds[1]);
+                    du[j / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                }
+                if (c == 0) {
+                    // P buffer pb is free once dV of step n - NP has run; dS
+                    // buffer db once dK and dQ of step n - 2 have.
+                    if (n >= C::NP && !warp_wait(bar(C::B_P_FREE + pb), ((n / C::NP) - 1) & 1, wd,
+                                                 ROLE_COMPUTE, blk_id)) {
+                        ok = false;
+                        break;
+                    }
+                    if (n >= 2 && !warp_wait(bar(C::B_DS_FREE + db), ((n / 2) - 1) & 1, wd,
+                                             ROLE_COMPUTE, blk_id)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                tmem_st16(tmem + lane_base + C::TM_P + pb * (BQ / 2) + col0 / 2, pu);
+                // dS row r, queries col0..col0+31, in the 128-byte-swizzled
+                // layout (16-byte chunk index XOR row % 8 inside 1 KiB atoms).
+                const uint32_t row_base = sds + (col0 / 64) * C::DS_SLAB + (r / 8) * 1024 +
+                                          (r % 8) * 128;
+                const int ch0 = (col0 % 64) / 8;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const uint32_t phys = uint32_t((ch0 + k4) ^ (r % 8));
+                    st_shared_v4(row_base + phys * 16, du[4 * k4], du[4 * k4 + 1], du[4 * k4 + 2],
+                                 du[4 * k4 + 3]);
+                }
+            }
+            if (!ok) break;
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(C::B_DS_READY + db));
+                mbar_arrive(bar(C::B_QD_EMPTY + s));
+            }
+        }
+        // Epilogue: dV and scale * dK of this warp's rows and column half.
+        if (ok && warp_wait(bar(C::B_ACC_FULL), 0, wd, ROLE_COMPUTE, blk_id)) {
+            tc_fence_after();
+            constexpr int HC = D / 2;                         // columns per half
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t tcol = (which == 0 ? C::TM_DV : C::TM_DK) + half * HC;
+                const float mul = which == 0 ? 1.f : scale;
+                __nv_bfloat16* dst = (which == 0 ? dv : dk) + ((long long)bh * N + key) * D + half * HC;
+#pragma unroll
+                for (int c = 0; c < HC / 32; ++c) {
+                    uint32_t x[32];
+                    tmem_ld32(tmem + lane_base + tcol + c * 32, x);
+                    if (key < N) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            uint4 w;
+                            w.x = pack_bf16x2(mul * __uint_as_float(x[8 * k4 + 0]),
+                                              mul * __uint_as_float(x[8 * k4 + 1]));
+                            w.y = pack_bf16x2(mul * __uint_as_float(x[8 * k4 + 2]),
+                                              mul * __uint_as_float(x[8 * k4 + 3]));
+                            w.z = pack_bf16x2(mul * __uint_as_float(x[8 * k4 + 4]),
+                                              mul * __uint_as_float(x[8 * k4 + 5]));
+                            w.w = pack_bf16x2(mul * __uint_as_float(x[8 * k4 + 6]),
+                                              mul * __uint_as_float(x[8 * k4 + 7]));
+                            d4[k4] = w;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    __syncwarp();          // single-lane roles rejoin their warps before the aligned barrier
+    tc_fence_before();
+    cta_sync();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+long long npad_of(int N) { return ((long long)N + BK - 1) / BK * BK; }
+
+struct WsLayout {
+    size_t dq_acc, lse2, dvec, total;
+};
+
+WsLayout ws_layout(long long BH, int N, int d) {
+    const long long np = npad_of(N);
+    WsLayout w;
+    w.dq_acc = 0;
+    w.lse2 = size_t(BH * np * d * 4);
+    w.dvec = w.lse2 + size_t(BH * np * 4);
+    w.total = w.dvec + size_t(BH * np * 4);
+    return w;
+}
+
+template <int D>
+fa_status launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int causal,
+                 float scale, unsigned char* ws, cudaStream_t stream, int dev,
+                 unsigned long long wd_ns) {
+    using C = Cfg<D>;
+    const long long BH = (long long)B * H;
+    const long long np = npad_of(N);
+    const WsLayout wl = ws_layout(BH, N, D);
+    float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_acc);
+    float* lse2 = reinterpret_cast<float*>(ws + wl.lse2);
+    float* dvec = reinterpret_cast<float*>(ws + wl.dvec);
+
+    const long long sb = (long long)H * N * D, sh = (long long)N * D, sn = D;
+    CUtensorMap mq, mk, mv, mdo;
+    if (fa_internal::encode_bhnd_map(&mq, q, D, N, H, B, sb, sh, sn, C::BQ) != FA_OK ||
+        fa_internal::encode_bhnd_map(&mk, k, D, N, H, B, sb, sh, sn, BK) != FA_OK ||
+        fa_internal::encode_bhnd_map(&mv, v, D, N, H, B, sb, sh, sn, BK) != FA_OK ||
+        fa_internal::encode_bhnd_map(&mdo, dout, D, N, H, B, sb, sh, sn, C::BQ) != FA_OK)
+        return FA_ERR_UNSUPPORTED;
+
+    // Per-device, idempotent and cheap; set on every call so a device switch
+    // between calls is covered.
+    (void)dev;
+    cudaError_t e = cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::ALLOC);
+    if (e != cudaSuccess) {
+        fa_internal::set_last_cuda_error(int(e));
+        return FA_ERR_LAUNCH;
+    }
+
+    const long long prep_threads = BH * np * (D / 8);
+    bwd_prep<D><<<unsigned((prep_threads + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
+        dvec, dq_acc, BH, N, int(np));
+    const long long nkb = (N + BK - 1) / BK;
+    bwd_kernel<D><<<unsigned(nkb * BH), NUM_THREADS, C::ALLOC, stream>>>(
+        mq, mk, mv, mdo, lse2, dvec, dq_acc, static_cast<__nv_bfloat16*>(dk),
+        static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, wd_ns);
+    const long long out_threads = BH * N * (D / 8);
+    bwd_dq_out<D><<<unsigned((out_threads + 255) / 256), 256, 0, stream>>>(
+        dq_acc, static_cast<__nv_bfloat16*>(dq), BH, N, int(np), scale);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        fa_internal::set_last_cuda_error(int(e));
+        return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace bwd
+
+int fa_internal::take_bwd_status(unsigned* word) {
+    unsigned w = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&w, bwd::g_bwd_status, sizeof(w));
+    const unsigned zero = 0;
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(bwd::g_bwd_status, &zero, sizeof(zero));
+    *word = w;
+    return int(e);
+}
+
+extern "C" {
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    if ((long long)B * H > 0x7fffffffLL || N > (1 << 30)) return 0;
+    return bwd::ws_layout((long long)B * H, N, d).total;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    using bwd::aligned;
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
+        return FA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    const long long BH = (long long)B * H;
+    if (BH > 0x7fffffffLL || N > (1 << 30)) return FA_ERR_UNSUPPORTED;
+    // One CTA per (key block, batch x head): the grid is a 1-D unsigned count.
+    if ((((long long)N + bwd::BK - 1) / bwd::BK) * BH > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    if (workspace_bytes < bwd::ws_layout(BH, N, d).total) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(lse, 4) || !aligned(workspace, 256))
+        return FA_ERR_MISALIGNED;
+
+    int dev = -1, sm_count = 0;
+    const int ds = fa_internal::current_device(&dev, &sm_count);
+    if (ds != FA_OK) return static_cast<fa_status>(ds);
+    const unsigned long long wd_ns = 4000ull * 1000000ull;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    if (d == 64)
+        return bwd::launch<64>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, ws, s,
+                                  dev, wd_ns);
+    return bwd::launch<128>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, ws, s,
+                               dev, wd_ns);
+}
+
+}  // extern "C"

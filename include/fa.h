@@ -207,6 +207,48 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
                         int num_splits, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_bwd_workspace_bytes -- device workspace fa_bwd needs for these sizes:
+ * an fp32 dQ accumulator [B][H][Npad][d] and two fp32 per-row vectors
+ * [B][H][Npad], Npad = N rounded up to a multiple of 128.  Returns 0 for
+ * sizes fa_bwd would reject.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * fa_bwd -- gradients of exact attention by recomputation.
+ *
+ * For O = softmax(scale * Q K^T [+ causal mask]) V with upstream gradient
+ * dO = dL/dO, computes dQ, dK, dV without storing P: each P block is rebuilt
+ * on chip from Q, K and the forward's LSE, as the page "Flash attention
+ * optimization" describes in "Sizing a tile, and why the backward pass
+ * recomputes instead of storing" (only the O(N) row statistics are kept).
+ * With D_i = sum_t dO_it O_it and P = exp(scale Q K^T - LSE):
+ *   dV = P^T dO,  dS = P * (dO V^T - D),  dQ = scale dS K,  dK = scale dS^T Q.
+ *
+ *  q, k, v, o, dout : bf16 [B][H][N][d] contiguous (o and lse as returned by
+ *                     fa_fwd for the same q, k, v, causal and scale).
+ *  lse              : fp32 [B][H][N], natural-log units.
+ *  dq, dk, dv       : bf16 [B][H][N][d] contiguous, written.
+ *  workspace        : device memory owned by the caller, 256-byte aligned,
+ *                     >= fa_bwd_workspace_bytes(B, H, N, d) bytes; overwritten
+ *                     and must not be shared by calls that may run at the same
+ *                     time.  Nothing is allocated per call.
+ *  B, H, N, d, causal, scale : as fa_fwd.
+ * Products P and dS are rounded to bf16 before their tensor-core products;
+ * accumulation is fp32.  dQ is accumulated with floating-point atomic adds,
+ * so its low bits may differ from run to run; dK and dV are deterministic.
+ * Errors: FA_ERR_INVALID_ARG (NULL pointers, sizes < 1, bad causal or scale,
+ * workspace too small), FA_ERR_UNSUPPORTED (d not 64/128, sizes beyond the
+ * limits of fa_fwd, device not sm_100), FA_ERR_MISALIGNED (tensors not
+ * 16-byte aligned, lse not 4-byte aligned, workspace not 256-byte aligned),
+ * FA_ERR_NO_DEVICE, FA_ERR_LAUNCH.  A watchdog timeout inside the kernel is
+ * reported by fa_get_device_status.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_fwd_debug -- fa_fwd with the kernel watchdog exposed, for tests.
  *
  *  watchdog_ms : every wait inside the kernel gives up after this many

@@ -148,3 +148,12 @@ def draw_qkv(B: int, H: int, N: int, d: int, seed: int, qk_std: float = 1.0):
 
 def workload_qkv(w: Workload):
     return draw_qkv(w.B, w.H, w.N, w.d, w.seed, w.qk_std)
+
+
+def draw_dout(B: int, H: int, N: int, d: int, seed: int):
+    """Seeded upstream gradient dO for the backward pass: standard normals of
+    shape (B, H, N, d) from a generator seeded with ``seed + 5000`` (so it
+    differs from the Q, K, V draw of the same seed), rounded to bf16."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed + 5000)
+    return torch.randn((B, H, N, d), generator=g, dtype=torch.float32).to(torch.bfloat16)

@@ -152,3 +152,32 @@ def test_decode_argument_validation_and_workspace_size():
     assert fa.decode_workspace_bytes(2, 3, 4, 1000, 128, 300) == 0
     assert fa.decode_workspace_bytes(2, 3, 4, 1000, 128, 0) > 0
     assert fa.fa_fwd_decode_raw(*ok) == fa.FA_ERR_NO_DEVICE                  # valid: stops at the device query
+
+
+def test_bwd_argument_validation_and_workspace_size():
+    W = 1 << 22
+    ok = [P, P, P, P, P, P, P, P, P, 2, 3, 1000, 128, 1, 0.1, W, 1 << 30, 0]
+    assert fa.fa_bwd_raw(*ok) == fa.FA_ERR_NO_DEVICE                         # valid: stops at the device query
+    for i in range(9):                                                        # any NULL tensor
+        a = list(ok); a[i] = 0
+        assert fa.fa_bwd_raw(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok); a[15] = 0
+    assert fa.fa_bwd_raw(*a) == fa.FA_ERR_INVALID_ARG                        # NULL workspace
+    a = list(ok); a[16] = fa.bwd_workspace_bytes(2, 3, 1000, 128) - 1
+    assert fa.fa_bwd_raw(*a) == fa.FA_ERR_INVALID_ARG                        # workspace too small
+    a = list(ok); a[13] = 2
+    assert fa.fa_bwd_raw(*a) == fa.FA_ERR_INVALID_ARG                        # causal flag
+    a = list(ok); a[14] = -1.0
+    assert fa.fa_bwd_raw(*a) == fa.FA_ERR_INVALID_ARG                        # scale
+    a = list(ok); a[12] = 96
+    assert fa.fa_bwd_raw(*a) == fa.FA_ERR_UNSUPPORTED                        # d = 96
+    a = list(ok); a[4] = P + 2
+    assert fa.fa_bwd_raw(*a) == fa.FA_ERR_MISALIGNED                         # dout alignment
+    a = list(ok); a[5] = P + 2
+    assert fa.fa_bwd_raw(*a) == fa.FA_ERR_MISALIGNED                         # lse alignment
+    a = list(ok); a[15] = W + 128
+    assert fa.fa_bwd_raw(*a) == fa.FA_ERR_MISALIGNED                         # workspace alignment
+    # workspace: fp32 dQ accumulator and two fp32 row vectors over N rounded up to 128
+    assert fa.bwd_workspace_bytes(2, 3, 1000, 128) == 6 * 1024 * 128 * 4 + 2 * 6 * 1024 * 4
+    assert fa.bwd_workspace_bytes(2, 3, 1000, 96) == 0
+    assert fa.bwd_workspace_bytes(0, 3, 1000, 64) == 0
