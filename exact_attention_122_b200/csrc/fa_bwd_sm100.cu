@@ -62,7 +62,11 @@ constexpr int COMPUTE_WARPS = 8;
 constexpr int DQ_WARP0 = 8;
 constexpr int MMA_WARP = 12;
 constexpr int TMA_WARP = 13;
-constexpr int NS = 2;               // Q / dO ring stages
+// Q / dO ring stages.  A stage is held from its load until block i's
+// gradient MMAs have run, about two steps; with two stages the next load's
+// latency was exposed on every step (measured on B200: three stages 24 %
+// faster on the 8K causal workload).
+constexpr int NS = 3;
 constexpr float LOG2E = 1.4426950408889634f;
 
 enum : uint32_t { ROLE_COMPUTE = 1u, ROLE_MMA = 2u, ROLE_PRODUCER = 3u, ROLE_DQ = 4u,
@@ -204,15 +208,18 @@ __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float
 }
 
 // ---------------------------------------------------------------------------
-// Pre-pass: D_i = dO_i . O_i (fp32), LSE2_i = LSE_i log2(e), zero dQ_acc.
-// Rows r in [N, Npad) get D = 0 and LSE2 = +inf.  D / 8 threads per row, each
+// Pre-pass: -D_i = -(dO_i . O_i) (fp32), -LSE2_i = -LSE_i log2(e), zero
+// dQ_acc.  Rows r in [N, Npad) get -D = 0 and -LSE2 = -inf (so P = 0).
+// Both are stored negated so the compute warps add them with packed f32x2
+// fused multiply-adds.  D / 8 threads per row, each
 // on 8 consecutive elements.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict__ o,
                                                 const __nv_bfloat16* __restrict__ dout,
                                                 const float* __restrict__ lse,
-                                                float* __restrict__ lse2, float* __restrict__ dvec,
+                                                float* __restrict__ nlse2,
+                                                float* __restrict__ ndvec,
                                                 float* __restrict__ dq_acc, long long BH, int N,
                                                 int Npad) {
     constexpr int TPR = D / 8;                          // threads per row
@@ -244,8 +251,8 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict_
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (part == 0) {
-        dvec[row] = r < N ? acc : 0.f;
-        lse2[row] = r < N ? lse[bh * N + r] * LOG2E : INFINITY;
+        ndvec[row] = r < N ? -acc : 0.f;
+        nlse2[row] = r < N ? -lse[bh * N + r] * LOG2E : -INFINITY;
     }
 }
 
@@ -271,6 +278,53 @@ __global__ void __launch_bounds__(256) bwd_dq_out(const float* __restrict__ dq_a
     *reinterpret_cast<uint4*>(dq + row * D + part * 8) = out;
 }
 
+// P and dS for 32 query columns of one key row (this thread's TMEM lane):
+//   p = 2^(s * scale log2(e) - LSE2),  ds = p * (dP - D),
+// both rounded to bf16 pairs.  nl / nd point at -LSE2 and -D of the 32
+// columns (shared memory).  MASK: zero p where the query precedes the key
+// (causal), or the query or key is past N.  Pairs of columns go through the
+// packed f32x2 pipe.
+template <bool MASK>
+__device__ __forceinline__ void p_ds_chunk(const uint32_t (&sv)[32], const uint32_t (&dpv)[32],
+                                           const float* nl, const float* nd, float cs, int qi0,
+                                           int key, int N, int causal, uint32_t (&pu)[16],
+                                           uint32_t (&du)[16]) {
+    const uint64_t cs2 = f2_pack(cs, cs);
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(nl + j);
+        const float4 d4 = *reinterpret_cast<const float4*>(nd + j);
+        const uint64_t l01 = f2_pack(l4.x, l4.y), l23 = f2_pack(l4.z, l4.w);
+        const uint64_t d01 = f2_pack(d4.x, d4.y), d23 = f2_pack(d4.z, d4.w);
+        const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])),
+                                    cs2, l01);
+        const uint64_t x23 = f2_fma(
+            f2_pack(__uint_as_float(sv[j + 2]), __uint_as_float(sv[j + 3])), cs2, l23);
+        float x[4], p[4];
+        f2_unpack(x01, x[0], x[1]);
+        f2_unpack(x23, x[2], x[3]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            p[u] = ex2(x[u]);
+            if (MASK) {
+                const int qi = qi0 + j + u;
+                if ((causal && qi < key) || qi >= N || key >= N) p[u] = 0.f;
+            }
+        }
+        const uint64_t t01 = f2_add(
+            f2_pack(__uint_as_float(dpv[j]), __uint_as_float(dpv[j + 1])), d01);
+        const uint64_t t23 = f2_add(
+            f2_pack(__uint_as_float(dpv[j + 2]), __uint_as_float(dpv[j + 3])), d23);
+        float ds[4];
+        f2_unpack(f2_mul(f2_pack(p[0], p[1]), t01), ds[0], ds[1]);
+        f2_unpack(f2_mul(f2_pack(p[2], p[3]), t23), ds[2], ds[3]);
+        pu[j / 2] = pack_bf16x2(p[0], p[1]);
+        pu[j / 2 + 1] = pack_bf16x2(p[2], p[3]);
+        du[j / 2] = pack_bf16x2(ds[0], ds[1]);
+        du[j / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Main kernel
 // ---------------------------------------------------------------------------
@@ -278,7 +332,7 @@ template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-           const float* __restrict__ lse2, const float* __restrict__ dvec,
+           const float* __restrict__ nlse2, const float* __restrict__ ndvec,
            float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
            __nv_bfloat16* __restrict__ dv, int BH, int H, int N, int Npad, int causal,
            float scale, unsigned long long watchdog_ns) {
@@ -369,8 +423,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                                 sl * 64, q0, h, b, full);
                 }
                 const long long vrow = (long long)bh * Npad + q0;
-                bulk_load(sbase + C::OFF_VEC + s * C::VEC_BYTES, lse2 + vrow, BQ * 4, full);
-                bulk_load(sbase + C::OFF_VEC + s * C::VEC_BYTES + BQ * 4, dvec + vrow, BQ * 4,
+                bulk_load(sbase + C::OFF_VEC + s * C::VEC_BYTES, nlse2 + vrow, BQ * 4, full);
+                bulk_load(sbase + C::OFF_VEC + s * C::VEC_BYTES + BQ * 4, ndvec + vrow, BQ * 4,
                           full);
                 ++issued;
             }
@@ -573,27 +627,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     if (lane == 0) mbar_arrive(bar(C::B_SDP_FREE));
                 }
                 uint32_t pu[16], du[16];
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4*>(vl + col0 + j);
-                    const float4 d4 = *reinterpret_cast<const float4*>(vd + col0 + j);
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float p[4], ds[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        p[u] = ex2(fmaf(__uint_as_float(sv[j + u]), cs, -lv[u]));
-                        if (need_mask) {
-                            const int qi = q0 + col0 + j + u;
-                            if ((causal && qi < key) || qi >= N || key >= N) p[u] = 0.f;
-                        }
-                        ds[u] = p[u] * (__uint_as_float(dpv[j + u]) - dd[u]);
-                    }
-                    pu[j / 2] = pack_bf16x2(p[0], p[1]);
-                    pu[j / 2 + 1] = pack_bf16x2(p[2], p[3]);
-                    du[j / 2] = pack_bf16x2(ds[0], ds[1]);
-                    du[j / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
-                }
+                if (need_mask)
+                    p_ds_chunk<true>(sv, dpv, vl + col0, vd + col0, cs, q0 + col0, key, N, causal,
+                                     pu, du);
+                else
+                    p_ds_chunk<false>(sv, dpv, vl + col0, vd + col0, cs, q0 + col0, key, N, causal,
+                                      pu, du);
                 if (c == 0) {
                     // P buffer pb is free once dV of step n - NP has run; dS
                     // buffer db once dK and dQ of step n - 2 have.
@@ -681,16 +720,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 long long npad_of(int N) { return ((long long)N + BK - 1) / BK * BK; }
 
 struct WsLayout {
-    size_t dq_acc, lse2, dvec, total;
+    size_t dq_acc, nlse2, ndvec, total;
 };
 
 WsLayout ws_layout(long long BH, int N, int d) {
     const long long np = npad_of(N);
     WsLayout w;
     w.dq_acc = 0;
-    w.lse2 = size_t(BH * np * d * 4);
-    w.dvec = w.lse2 + size_t(BH * np * 4);
-    w.total = w.dvec + size_t(BH * np * 4);
+    w.nlse2 = size_t(BH * np * d * 4);
+    w.ndvec = w.nlse2 + size_t(BH * np * 4);
+    w.total = w.ndvec + size_t(BH * np * 4);
     return w;
 }
 
@@ -704,8 +743,8 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
     const long long np = npad_of(N);
     const WsLayout wl = ws_layout(BH, N, D);
     float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_acc);
-    float* lse2 = reinterpret_cast<float*>(ws + wl.lse2);
-    float* dvec = reinterpret_cast<float*>(ws + wl.dvec);
+    float* nlse2 = reinterpret_cast<float*>(ws + wl.nlse2);
+    float* ndvec = reinterpret_cast<float*>(ws + wl.ndvec);
 
     const long long sb = (long long)H * N * D, sh = (long long)N * D, sn = D;
     CUtensorMap mq, mk, mv, mdo;
@@ -727,11 +766,11 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
 
     const long long prep_threads = BH * np * (D / 8);
     bwd_prep<D><<<unsigned((prep_threads + 255) / 256), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
-        dvec, dq_acc, BH, N, int(np));
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, nlse2,
+        ndvec, dq_acc, BH, N, int(np));
     const long long nkb = (N + BK - 1) / BK;
     bwd_kernel<D><<<unsigned(nkb * BH), NUM_THREADS, C::ALLOC, stream>>>(
-        mq, mk, mv, mdo, lse2, dvec, dq_acc, static_cast<__nv_bfloat16*>(dk),
+        mq, mk, mv, mdo, nlse2, ndvec, dq_acc, static_cast<__nv_bfloat16*>(dk),
         static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, wd_ns);
     const long long out_threads = BH * N * (D / 8);
     bwd_dq_out<D><<<unsigned((out_threads + 255) / 256), 256, 0, stream>>>(
