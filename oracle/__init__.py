@@ -13,6 +13,7 @@ online softmax by hand".
 
 from .exact_attention import (  # noqa: F401
     bf16_bits_to_f64,
+    e4m3_bits_to_f64,
     attention_fp64,
     attention_bwd_fp64,
     attention_bwd_rows_fp64,

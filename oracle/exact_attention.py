@@ -59,6 +59,24 @@ def bf16_bits_to_f64(bits) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
+def e4m3_bits_to_f64(bits) -> np.ndarray:
+    """Exact value of FP8 E4M3 codes (uint8) as float64.
+
+    E4M3 (the "fn" variant: no infinities): 1 sign bit, 4 exponent bits with
+    bias 7, 3 mantissa bits.  Exponent field 0 is subnormal,
+    (-1)^s * 2^-6 * m/8; otherwise (-1)^s * 2^(e-7) * (1 + m/8).  The codes
+    0x7F and 0xFF (exponent and mantissa all ones) are NaN; 0x7E = 448 is the
+    largest finite value.
+    """
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    val = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64)))
+    val = sign * val
+    return np.where((b & 0x7F) == 0x7F, np.nan, val)
+
+
 def _as_f64(x) -> np.ndarray:
     """Accept a numpy array or a CPU torch tensor (any real dtype) -> float64."""
     if hasattr(x, "detach"):  # torch tensor: go through float32, exact for bf16/fp16/fp32

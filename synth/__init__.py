@@ -157,3 +157,37 @@ def draw_dout(B: int, H: int, N: int, d: int, seed: int):
     g = torch.Generator(device="cpu")
     g.manual_seed(seed + 5000)
     return torch.randn((B, H, N, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) inputs for the FP8 forward.  Per-tensor scaling: a tensor x is
+# stored as codes x8 = e4m3(x / s) with s = amax(|x|) / 448 (448 is the
+# largest finite E4M3 value), rounded to nearest even by torch's
+# float8_e4m3fn cast; its value is x8 * s.  Both the CUDA path and the
+# oracle consume the same codes and scales.
+# ---------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """(uint8 codes, float scale) of a float32 tensor, per-tensor scale."""
+    amax = float(x.abs().max())
+    scale = amax / E4M3_MAX if amax > 0 else 1.0
+    codes = (x / scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale
+
+
+def draw_qkv_fp8(B: int, H: int, N: int, d: int, seed: int, qk_std: float = 1.0):
+    """Seeded FP8 Q, K, V: the float32 draws of draw_qkv (same generator and
+    order), each quantized per tensor.  Returns ((q8, k8, v8), (sq, sk, sv))."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    shape = (B, H, N, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    if qk_std != 1.0:
+        q.mul_(qk_std)
+        k.mul_(qk_std)
+    (q8, sq), (k8, sk), (v8, sv) = quantize_e4m3(q), quantize_e4m3(k), quantize_e4m3(v)
+    return (q8, k8, v8), (sq, sk, sv)
