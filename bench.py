@@ -548,6 +548,63 @@ def run_bwd(args):
     return 0
 
 
+def run_fp8(args):
+    """FP8 forward of the workload's shape: one step = fa_fwd_fp8 (V^T pass and
+    the attention kernel) on E4M3 inputs already in device memory."""
+    import torch
+
+    import exact_attention_122_b200 as fa
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = synth.workload(args.workload)
+    (q8, k8, v8), (sq, sk, sv) = synth.draw_qkv_fp8(w.B, w.H, w.N, w.d, seed=w.seed,
+                                                     qk_std=w.qk_std)
+    q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
+    stream = torch.cuda.Stream(device=dev)
+    o = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fp8_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+
+    def step():
+        fa.fa_fwd_fp8(q8, k8, v8, sq, sk, sv, causal=w.causal, out=o, lse=lse, workspace=ws,
+                      stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clocks:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+    st, word = fa.device_status(stream.cuda_stream)
+    if st != fa.FA_OK:
+        raise SystemExit(f"kernel status {fa.status_string(st)} {word:#x}")
+    ms = e0.elapsed_time(e1) / args.steps
+    value = w.flops / (ms / 1e3) / 1e12
+    peak_bf16, _, peak_src = load_peaks()
+    # FP8 dense peak: the measured bf16 peak times the nominal FP8 / bf16 ratio (4.5 / 2.25).
+    peak = 2.0 * peak_bf16
+    line = {"metric": "attention fwd TFLOP/s, FP8 E4M3 inputs (1 GPU)", "value": value,
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": w.name + "_fp8", "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "causal": w.causal, "l2": "inputs 268 MB > 126 MB L2; no flush"},
+            "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s",
+                         "frac": value / peak, "traffic": None,
+                         "peak_source": f"{peak_src} bf16 x 2 (nominal FP8/bf16 ratio)",
+                         "kernel": "transpose_v_e4m3 + fa_fwd_kernel<128, 8, true> (whole step)"},
+            "gpu_launches": 3 * args.steps, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_sweep(args):
     import torch
 
@@ -608,6 +665,8 @@ def main(argv=None):
                          "on the long causal workloads) or fa_fwd (static)")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode-shaped path (HBM-bound) instead of the headline line")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the FP8 (E4M3) forward of the workload's shape")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward pass (fa_bwd) of the workload instead of the forward")
     ap.add_argument("--sweep", action="store_true",
@@ -621,6 +680,8 @@ def main(argv=None):
         return run_sweep(args)
     if args.bwd:
         return run_bwd(args)
+    if args.fp8:
+        return run_fp8(args)
     if args.decode:
         return run_decode(args)
     w = synth.workload(args.workload)

@@ -16,7 +16,7 @@ FA_ERR_NO_DEVICE = 6
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_dynamic_noalloc",
                     "fa_fwd_decode_workspace_bytes", "fa_fwd_decode", "fa_bwd_workspace_bytes",
-                    "fa_bwd", "fa_fwd_debug",
+                    "fa_bwd", "fa_fwd_fp8_workspace_bytes", "fa_fwd_fp8", "fa_fwd_debug",
                     "fa_get_device_status", "fa_status_string", "fa_last_cuda_error", "fa_version")
 DECODE_MAX_QUERIES = 16                # FA_DECODE_MAX_QUERIES
 DECODE_MAX_SPLITS = 256                # FA_DECODE_MAX_SPLITS
@@ -62,6 +62,11 @@ def library() -> ctypes.CDLL:
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp,
                            ctypes.c_size_t, vp]
     lib.fa_bwd.restype = i
+    lib.fa_fwd_fp8_workspace_bytes.argtypes = [i, i, i, i]
+    lib.fa_fwd_fp8_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, vp, ctypes.c_size_t,
+                               vp]
+    lib.fa_fwd_fp8.restype = i
     lib.fa_fwd_debug.argtypes = fwd_args + [u, i]
     lib.fa_fwd_debug.restype = i
     lib.fa_get_device_status.argtypes = [vp, ctypes.POINTER(u)]
@@ -225,6 +230,55 @@ def fa_bwd(q, k, v, out, lse, dout, causal: bool = False, scale: float | None = 
     if st != FA_OK:
         raise FaError(st, "fa_bwd")
     return dq, dk, dv
+
+
+def fp8_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(library().fa_fwd_fp8_workspace_bytes(B, H, N, d))
+
+
+def fa_fwd_fp8_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int,
+                   N: int, d: int, causal: int, scale: float, descale_q: float, descale_k: float,
+                   descale_v: float, ws_ptr: int, ws_bytes: int, stream_ptr: int) -> int:
+    """Direct call of fa_fwd_fp8; returns the fa_status code."""
+    return library().fa_fwd_fp8(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal, scale,
+                                descale_q, descale_k, descale_v, ws_ptr, ws_bytes, stream_ptr)
+
+
+def fa_fwd_fp8(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float,
+               causal: bool = False, scale: float | None = None, out=None, lse=None,
+               workspace=None, stream=None):
+    """O (bf16), LSE of attention over FP8 E4M3 inputs: q8, k8, v8 contiguous
+    CUDA tensors (B, H, N, 128) of dtype uint8 or torch.float8_e4m3fn holding
+    the codes; the values are code * descale_x.  ``workspace`` (at least
+    fp8_workspace_bytes(B, H, N, d) bytes) is allocated with torch when not
+    given."""
+    import torch
+
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        if not (t.is_cuda and t.element_size() == 1 and t.dim() == 4 and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous one-byte CUDA tensor")
+    B, H, N, d = q8.shape
+    if k8.shape != q8.shape or v8.shape != q8.shape:
+        raise ValueError("q8, k8 and v8 must have one shape (B, H, N, d)")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    need = fp8_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q8.device)
+    with torch.cuda.device(q8.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q8.device)
+        st = fa_fwd_fp8_raw(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
+                            lse.data_ptr(), B, H, N, d, 1 if causal else 0, float(scale),
+                            float(descale_q), float(descale_k), float(descale_v),
+                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            s.cuda_stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_fp8")
+    return out, lse
 
 
 _WORKSPACES = {}

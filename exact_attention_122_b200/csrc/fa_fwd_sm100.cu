@@ -96,11 +96,18 @@ enum : uint32_t {
     ROLE_SOFTMAX = 1u, ROLE_MMA = 2u, ROLE_PRODUCER = 3u, ROLE_DRAIN = 4u
 };
 
-template <int D, int NS>
+// F8: Q, K, V are FP8 E4M3 (one byte per element) and V arrives transposed
+// (d rows x keys), so every operand is K-major; a 128-byte swizzled row then
+// holds 128 elements instead of 64.
+template <int D, int NS, bool F8 = false>
 struct Layout {
-    static constexpr int Q_BYTES = BM * D * 2;       // one sub-tile of Q
-    static constexpr int KV_BYTES = BN * D * 2;      // one K or V tile
-    static constexpr int HALF_BYTES = BM * SW_COLS * 2;  // one 64-column slab (16 KiB)
+    static constexpr int EB = F8 ? 1 : 2;            // bytes per element
+    static constexpr int Q_BYTES = BM * D * EB;      // one sub-tile of Q
+    static constexpr int KV_BYTES = BN * D * EB;     // one K or V tile
+    static constexpr int HALF_BYTES = BM * 128;      // one 128-byte-wide slab (16 KiB)
+    static constexpr int SLABS = D * EB / 128;       // slabs per Q / K tile
+    static constexpr int SLAB_ELEMS = 128 / EB;      // elements per slab row
+    static constexpr int QK_STEPS = D * EB / 32;     // 32-byte K steps of S = Q K^T
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = 2 * Q_BYTES;
     static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
@@ -226,36 +233,53 @@ __device__ __forceinline__ Unit decode_unit(int i, int BH, int N, int causal, in
 // S = Q K^T for one sub-tile: M=128 query rows, N=128 keys, K=d in steps
 // of 16.  Both operands K-major with 128-byte swizzle: a step is 32 bytes
 // inside a swizzled row, and 64-column slabs are HALF_BYTES apart.
-template <int D, int HALF_BYTES>
+// A step is 16 bf16 or 32 FP8 elements: 32 bytes either way.
+template <int STEPS, int HALF_BYTES, bool F8>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc,
                                          uint32_t idesc) {
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
+    for (int kk = 0; kk < STEPS; ++kk) {
         const uint32_t off = uint32_t(((kk / 4) * HALF_BYTES + (kk % 4) * 32) >> 4);
-        mma_ss(d_tmem, desc_add(q_desc, off), desc_add(k_desc, off), idesc, kk > 0 ? 1u : 0u);
+        if constexpr (F8)
+            mma_ss_f8(d_tmem, desc_add(q_desc, off), desc_add(k_desc, off), idesc, kk > 0 ? 1u : 0u);
+        else
+            mma_ss(d_tmem, desc_add(q_desc, off), desc_add(k_desc, off), idesc, kk > 0 ? 1u : 0u);
     }
 }
 
-// O += P V for one sub-tile: A = P from TMEM (16 keys = 8 columns of bf16
-// pairs per step), B = V MN-major (16 key rows of 128 bytes per step).
+// O += P V for one sub-tile: A = P from TMEM (8 columns per step: 16 keys
+// as bf16 pairs, or 32 keys as FP8 quads).  bf16: B = V MN-major, 16 key
+// rows of 128 bytes per step.  FP8: B = V^T K-major (d rows of 128 keys), a
+// step is 32 bytes inside the swizzled rows.
+template <bool F8>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc,
                                          uint32_t idesc, bool first) {
+    if constexpr (F8) {
 #pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk) {
-        const uint32_t off = uint32_t((kk * 16 * 128) >> 4);
-        mma_ts(o_tmem, p_tmem + kk * 8, desc_add(v_desc, off), idesc, (first && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < BN / 32; ++kk)
+            mma_ts_f8(o_tmem, p_tmem + kk * 8, desc_add(v_desc, uint32_t((kk * 32) >> 4)), idesc,
+                      (first && kk == 0) ? 0u : 1u);
+    } else {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint32_t off = uint32_t((kk * 16 * 128) >> 4);
+            mma_ts(o_tmem, p_tmem + kk * 8, desc_add(v_desc, off), idesc,
+                   (first && kk == 0) ? 0u : 1u);
+        }
     }
 }
 
 // P = 2^(s * scale_log2 - m) for one score row held in registers, written
-// to TMEM as bf16 pairs over the row's first 64 columns; the row sum goes to
+// to TMEM over the row's first columns: bf16 pairs (64 columns) or, with F8,
+// FP8 E4M3 quads (32 columns).  The row sum (of the unrounded fp32 P) goes to
 // four packed partial accumulators.  The first NPOLY columns of every
 // 32-column chunk use exp2_poly, the rest MUFU ex2.
-template <int NPOLY>
+template <int NPOLY, bool F8 = false>
 __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_log2, float neg_m,
                                              uint64_t (&acc)[4], uint32_t tS) {
     const uint64_t c2 = f2_pack(scale_log2, scale_log2);
     const uint64_t m2 = f2_pack(neg_m, neg_m);
+    uint64_t pf_prev = 0;                        // F8: the previous pair of P values
 #pragma unroll
     for (int c = 0; c < BN / 32; ++c) {
         uint32_t pk[16];
@@ -272,23 +296,40 @@ __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_l
                 p1 = ex2(x1);
             }
             acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-            pk[i] = pack_bf16x2(p0, p1);
+            if constexpr (F8) {
+                // keys 2i-2 .. 2i+1 go into word i/2 once both pairs exist
+                if (i & 1) {
+                    float q0, q1;
+                    f2_unpack(pf_prev, q0, q1);
+                    pk[i / 2] = pack_e4m3x4(q0, q1, p0, p1);
+                } else {
+                    pf_prev = f2_pack(p0, p1);
+                }
+            } else {
+                pk[i] = pack_bf16x2(p0, p1);
+            }
         }
-        tmem_st16(tS + c * 16, pk);              // P (bf16) over S columns [0, 64)
+        if constexpr (F8)
+            tmem_st8(tS + c * 8, pk);            // P (FP8) over S columns [0, 32)
+        else
+            tmem_st16(tS + c * 16, pk);          // P (bf16) over S columns [0, 64)
     }
 }
 
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <int D, int NS>
+// F8: Q, K and V^T are E4M3 (tmV then maps V^T, d rows x keys); scale_log2
+// includes the Q and K dequantisation scales and o_scale (V's scale)
+// multiplies O in the epilogue.  Unused (1) in the bf16 kernel.
+template <int D, int NS, bool F8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ Og,
                   float* __restrict__ LSEg, int BH, int H, int N, int causal, float scale_log2,
                   int hg, long long o_sb, long long o_sh, long long o_sn, int* __restrict__ sched,
-                  unsigned long long watchdog_ns, int inject) {
-    using L = Layout<D, NS>;
+                  unsigned long long watchdog_ns, int inject, float o_scale) {
+    using L = Layout<D, NS, F8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -407,9 +448,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 mbar_arrive_expect_tx(bar(L::B_Q_FULL), 2 * L::Q_BYTES);
                 for (int t = 0; t < 2; ++t)
-                    for (int h = 0; h < D / SW_COLS; ++h)
-                        tma_load_4d(sQ + t * L::Q_BYTES + h * L::HALF_BYTES, &tmQ, h * SW_COLS,
-                                    w.r0 + t * BM, wh, wb, bar(L::B_Q_FULL));
+                    for (int h = 0; h < L::SLABS; ++h)
+                        tma_load_4d(sQ + t * L::Q_BYTES + h * L::HALF_BYTES, &tmQ,
+                                    h * L::SLAB_ELEMS, w.r0 + t * BM, wh, wb, bar(L::B_Q_FULL));
                 ++q_issued;
                 for (int j = 0; j < w.nb1 && ok; ++j) {
                     for (int kind = 0; kind < 2; ++kind) {
@@ -424,10 +465,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             skipped = true;  // fault injection: this copy is never issued
                         } else {
                             mbar_arrive_expect_tx(bar(L::B_KV_FULL + s), L::KV_BYTES);
-                            const CUtensorMap* map = kind == 0 ? &tmK : &tmV;
-                            for (int h = 0; h < D / SW_COLS; ++h)
-                                tma_load_4d(sKV + s * L::KV_BYTES + h * L::HALF_BYTES, map,
-                                            h * SW_COLS, j * BN, wh, wb, bar(L::B_KV_FULL + s));
+                            if (F8 && kind == 1) {
+                                // V^T tile: all d rows, keys j*BN .. j*BN+127
+                                tma_load_4d(sKV + s * L::KV_BYTES, &tmV, j * BN, 0, wh, wb,
+                                            bar(L::B_KV_FULL + s));
+                            } else {
+                                const CUtensorMap* map = kind == 0 ? &tmK : &tmV;
+                                for (int h = 0; h < L::SLABS; ++h)
+                                    tma_load_4d(sKV + s * L::KV_BYTES + h * L::HALF_BYTES, map,
+                                                h * L::SLAB_ELEMS, j * BN, wh, wb,
+                                                bar(L::B_KV_FULL + s));
+                            }
                         }
                         ++fills;
                     }
@@ -457,8 +505,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // overwrites it, and a commit after S_t also covers the PV before it.
         // ------------------------------------------------------------------
         if (lane == 0) {
-            constexpr uint32_t ID_S = idesc_bf16(BM, BN, false);
-            constexpr uint32_t ID_PV = idesc_bf16(BM, D, true);
+            constexpr uint32_t ID_S = F8 ? idesc_e4m3(BM, BN) : idesc_bf16(BM, BN, false);
+            constexpr uint32_t ID_PV = F8 ? idesc_e4m3(BM, D) : idesc_bf16(BM, D, true);
             uint32_t cons = 0, units = 0, pcnt0 = 0, pcnt1 = 0;
             bool ok = true;
             bool issued = false;
@@ -468,7 +516,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
             const uint64_t dq1 = sdesc_sw128(sQ + L::Q_BYTES, 16, 1024);
             const uint64_t dk0 = sdesc_sw128(sKV, 16, 1024);
-            const uint64_t dv0 = sdesc_sw128(sKV, L::HALF_BYTES, 1024);
+            const uint64_t dv0 = F8 ? sdesc_sw128(sKV, 16, 1024)     // V^T: K-major
+                                    : sdesc_sw128(sKV, L::HALF_BYTES, 1024);
             const uint32_t stage_step = uint32_t(L::KV_BYTES >> 4);
             const uint32_t tS0 = tmem + L::TM_S0, tS1 = tmem + L::TM_S1;
             const uint32_t tO0 = tmem + L::TM_O0, tO1 = tmem + L::TM_O1;
@@ -483,9 +532,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 }
                 ++cons;
-                issue_qk<D, L::HALF_BYTES>(tS0, dq0, desc_add(dk0, sK * stage_step), ID_S);
+                issue_qk<L::QK_STEPS, L::HALF_BYTES, F8>(tS0, dq0, desc_add(dk0, sK * stage_step), ID_S);
                 tc_commit(bar(L::B_S_FULL + 0));
-                issue_qk<D, L::HALF_BYTES>(tS1, dq1, desc_add(dk0, sK * stage_step), ID_S);
+                issue_qk<L::QK_STEPS, L::HALF_BYTES, F8>(tS1, dq1, desc_add(dk0, sK * stage_step), ID_S);
                 tc_commit(bar(L::B_S_FULL + 1));
                 tc_commit(bar(L::B_KV_EMPTY + sK));
                 issued = true;
@@ -518,9 +567,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         }
                         ++pcnt0;
                         tc_fence_after();
-                        issue_pv(tO0, tS0, desc_add(dv0, sV * stage_step), ID_PV, j == 0);
+                        issue_pv<F8>(tO0, tS0, desc_add(dv0, sV * stage_step), ID_PV, j == 0);
                         if (j + 1 < w.nb0) {
-                            issue_qk<D, L::HALF_BYTES>(tS0, dq0, desc_add(dk0, sK * stage_step), ID_S);
+                            issue_qk<L::QK_STEPS, L::HALF_BYTES, F8>(tS0, dq0, desc_add(dk0, sK * stage_step), ID_S);
                             tc_commit(bar(L::B_S_FULL + 0));
                         }
                         if (j == w.nb0 - 1) tc_commit(bar(L::B_O_FULL + 0));
@@ -535,9 +584,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     ++pcnt1;
                     tc_fence_after();
-                    issue_pv(tO1, tS1, desc_add(dv0, sV * stage_step), ID_PV, j == 0);
+                    issue_pv<F8>(tO1, tS1, desc_add(dv0, sV * stage_step), ID_PV, j == 0);
                     if (next) {
-                        issue_qk<D, L::HALF_BYTES>(tS1, dq1, desc_add(dk0, sK * stage_step), ID_S);
+                        issue_qk<L::QK_STEPS, L::HALF_BYTES, F8>(tS1, dq1, desc_add(dk0, sK * stage_step), ID_S);
                         tc_commit(bar(L::B_S_FULL + 1));
                     }
                     tc_commit(bar(L::B_KV_EMPTY + sV));
@@ -647,9 +696,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // Tiles without masked scores may use the FMA-pipe 2^x for
                 // part of the row; the choice is warp-uniform, made once.
                 if (POLY_COLS > 0 && !(tail || diag))
-                    exp_row_to_p<POLY_COLS>(s, scale_log2, neg_m, acc, tS);
+                    exp_row_to_p<POLY_COLS, F8>(s, scale_log2, neg_m, acc, tS);
                 else
-                    exp_row_to_p<0>(s, scale_log2, neg_m, acc, tS);
+                    exp_row_to_p<0, F8>(s, scale_log2, neg_m, acc, tS);
                 {
                     float a0, a1, a2, a3, a4, a5, a6, a7;
                     f2_unpack(acc[0], a0, a1);
@@ -668,7 +717,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ++ocnt;
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
-            const float inv_l = 1.f / l;
+            float inv_l = 1.f / l;
+            if constexpr (F8) inv_l *= o_scale;
             const bool store = row < N;
             const int wb = w.bh / H, wh = w.bh - (w.bh / H) * H;     // batch, head
             __nv_bfloat16* orow = Og + wb * o_sb + wh * o_sh + (long long)(store ? row : 0) * o_sn;
@@ -738,18 +788,18 @@ DeviceInfo g_dev[MAX_DEVICES];
 std::once_flag g_encode_once;
 EncodeTiledFn g_encode = nullptr;
 
-template <int D, int NS>
+template <int D, int NS, bool F8>
 struct Instance {
     static std::once_flag once[MAX_DEVICES];
     static cudaError_t attr_err[MAX_DEVICES];
     static int regs[MAX_DEVICES];
 };
-template <int D, int NS>
-std::once_flag Instance<D, NS>::once[MAX_DEVICES];
-template <int D, int NS>
-cudaError_t Instance<D, NS>::attr_err[MAX_DEVICES];
-template <int D, int NS>
-int Instance<D, NS>::regs[MAX_DEVICES];
+template <int D, int NS, bool F8>
+std::once_flag Instance<D, NS, F8>::once[MAX_DEVICES];
+template <int D, int NS, bool F8>
+cudaError_t Instance<D, NS, F8>::attr_err[MAX_DEVICES];
+template <int D, int NS, bool F8>
+int Instance<D, NS, F8>::regs[MAX_DEVICES];
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -897,34 +947,32 @@ long long choose_head_group(long long BH, int N, int D, int causal, int grid) {
     return best;
 }
 
-template <int D, int NS>
-fa_status launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                 int N, const Strides3 (&st)[4], int causal, float scale, int* sched,
-                 cudaStream_t stream, int dev, unsigned long long watchdog_ns, int inject) {
-    using L = fa::Layout<D, NS>;
-    auto kern = fa::fa_fwd_kernel<D, NS>;
-    std::call_once(Instance<D, NS>::once[dev], [&] {
-        Instance<D, NS>::attr_err[dev] =
+// Launches fa_fwd_kernel<D, NS, F8> on prepared tensor maps: per-device
+// attribute setup, head-group choice, dynamic-schedule counter reset.
+template <int D, int NS, bool F8>
+fa_status launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        void* o, float* lse, int B, int H, int N, const Strides3& ost, int causal,
+                        float scale_log2, float o_scale, int* sched, cudaStream_t stream, int dev,
+                        unsigned long long watchdog_ns, int inject) {
+    using L = fa::Layout<D, NS, F8>;
+    using I = Instance<D, NS, F8>;
+    auto kern = fa::fa_fwd_kernel<D, NS, F8>;
+    std::call_once(I::once[dev], [&] {
+        I::attr_err[dev] =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
         cudaFuncAttributes fa_attr;
-        if (Instance<D, NS>::attr_err[dev] == cudaSuccess &&
-            cudaFuncGetAttributes(&fa_attr, kern) == cudaSuccess)
-            Instance<D, NS>::regs[dev] = fa_attr.numRegs;
+        if (I::attr_err[dev] == cudaSuccess && cudaFuncGetAttributes(&fa_attr, kern) == cudaSuccess)
+            I::regs[dev] = fa_attr.numRegs;
     });
-    if (Instance<D, NS>::attr_err[dev] != cudaSuccess) {
-        t_last_cuda_error = int(Instance<D, NS>::attr_err[dev]);
+    if (I::attr_err[dev] != cudaSuccess) {
+        t_last_cuda_error = int(I::attr_err[dev]);
         return FA_ERR_LAUNCH;
     }
     // The setmaxnreg split was sized for REGS_LAUNCH registers per thread;
     // with any other launch allocation setmaxnreg.inc could wait forever,
     // so such a build is refused rather than launched.
-    if (Instance<D, NS>::regs[dev] != fa::REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
+    if (I::regs[dev] != fa::REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
     const long long BH = (long long)B * H;
-    CUtensorMap mq, mk, mv;
-    if (encode_map(&mq, q, D, N, H, B, st[0]) != FA_OK ||
-        encode_map(&mk, k, D, N, H, B, st[1]) != FA_OK ||
-        encode_map(&mv, v, D, N, H, B, st[2]) != FA_OK)
-        return FA_ERR_UNSUPPORTED;
     const long long nq2 = (N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
     const long long units = nq2 * BH;
     const int grid = int(units < g_dev[dev].sm_count ? units : g_dev[dev].sm_count);
@@ -932,14 +980,13 @@ fa_status launch(const void* q, const void* k, const void* v, void* o, float* ls
     // schedule: CTAs claim units greedily, so balance no longer depends on the
     // group size; groups then hold about 16 MiB of K/V (all heads when the
     // whole K/V fits in 32 MiB).
-    const long long kv_head_bytes = 2LL * N * D * 2;
+    const long long kv_head_bytes = 2LL * N * D * L::EB;
     long long hg = sched ? ((BH * kv_head_bytes <= (32LL << 20)) ? BH : (16LL << 20) / kv_head_bytes)
                          : choose_head_group(BH, N, D, causal, grid);
 #ifdef FA_HEAD_GROUP
     hg = FA_HEAD_GROUP;
 #endif
     hg = hg < 1 ? 1 : (hg > BH ? BH : hg);
-    const float scale_log2 = scale * 1.4426950408889634f;
     if (sched) {
         const cudaError_t me = cudaMemsetAsync(sched, 0, sizeof(int), stream);
         if (me != cudaSuccess) {
@@ -949,14 +996,88 @@ fa_status launch(const void* q, const void* k, const void* v, void* o, float* ls
     }
     kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o),
                                                      lse, int(BH), H, N, causal, scale_log2,
-                                                     int(hg), st[3].b, st[3].h, st[3].n, sched,
-                                                     watchdog_ns, inject);
+                                                     int(hg), ost.b, ost.h, ost.n, sched,
+                                                     watchdog_ns, inject, o_scale);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         t_last_cuda_error = int(e);
         return FA_ERR_LAUNCH;
     }
     return FA_OK;
+}
+
+template <int D, int NS>
+fa_status launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, const Strides3 (&st)[4], int causal, float scale, int* sched,
+                 cudaStream_t stream, int dev, unsigned long long watchdog_ns, int inject) {
+    CUtensorMap mq, mk, mv;
+    if (encode_map(&mq, q, D, N, H, B, st[0]) != FA_OK ||
+        encode_map(&mk, k, D, N, H, B, st[1]) != FA_OK ||
+        encode_map(&mv, v, D, N, H, B, st[2]) != FA_OK)
+        return FA_ERR_UNSUPPORTED;
+    const float scale_log2 = scale * 1.4426950408889634f;
+    return launch_kernel<D, NS, false>(mq, mk, mv, o, lse, B, H, N, st[3], causal, scale_log2, 1.f,
+                                       sched, stream, dev, watchdog_ns, inject);
+}
+
+// ---------------------------------------------------------------------------
+// FP8 forward: V^T pre-pass, E4M3 tensor maps, kernel launch.
+// ---------------------------------------------------------------------------
+constexpr int FP8_D = 128;
+constexpr int FP8_NS = 8;                        // 16 KiB K or V^T tiles: 8 ring stages
+
+long long fp8_npad(int N) { return ((long long)N + fa::BN - 1) / fa::BN * fa::BN; }
+
+// V [BH][N][D] -> V^T [BH][D][Npad] (keys n >= N zero), one 64-key block of
+// one (batch, head) per CTA, through a shared-memory tile.
+template <int D>
+__global__ void __launch_bounds__(256) transpose_v_e4m3(const uint8_t* __restrict__ v,
+                                                        uint8_t* __restrict__ vt, int N,
+                                                        long long Npad) {
+    __shared__ __align__(16) uint8_t tile[64][D + 16];
+    const long long bh = blockIdx.y;
+    const int k0 = blockIdx.x * 64;
+    const uint8_t* src = v + bh * (long long)N * D;
+    for (int i = threadIdx.x; i < 64 * D / 16; i += 256) {
+        const int r = i / (D / 16), c = i % (D / 16);
+        uint4 x = make_uint4(0u, 0u, 0u, 0u);
+        if (k0 + r < N) x = *reinterpret_cast<const uint4*>(src + (long long)(k0 + r) * D + c * 16);
+        *reinterpret_cast<uint4*>(&tile[r][c * 16]) = x;
+    }
+    __syncthreads();
+    uint8_t* dst = vt + bh * D * Npad;
+    for (int i = threadIdx.x; i < D * 4; i += 256) {
+        const int dr = i / 4, kc = i % 4;            // d row, 16-key chunk
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int k = kc * 16 + 4 * q;
+            w[q] = uint32_t(tile[k][dr]) | (uint32_t(tile[k + 1][dr]) << 8) |
+                   (uint32_t(tile[k + 2][dr]) << 16) | (uint32_t(tile[k + 3][dr]) << 24);
+        }
+        *reinterpret_cast<uint4*>(dst + (long long)dr * Npad + k0 + kc * 16) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// 4-D E4M3 tensor map (inner, rows, H, B), contiguous, byte strides; box
+// (128, box_rows, 1, 1) in 128-byte swizzle.
+fa_status encode_map_e4m3(CUtensorMap* map, const void* base, long long inner, long long rows,
+                          int H, int B, int box_rows) {
+    const cuuint64_t dims[4] = {cuuint64_t(inner), cuuint64_t(rows), cuuint64_t(H), cuuint64_t(B)};
+    const cuuint64_t strides[3] = {cuuint64_t(inner), cuuint64_t(inner * rows),
+                                   cuuint64_t(inner * rows * H)};
+    const cuuint32_t box[4] = {128u, cuuint32_t(box_rows), 1u, 1u};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+size_t fp8_workspace_bytes(long long BH, int N) {
+    return size_t(FA_DYNAMIC_WORKSPACE_BYTES) + size_t(BH * FP8_D * fp8_npad(N));
 }
 
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -1092,6 +1213,50 @@ fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, vo
     // before the kernel runs.
     return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale,
                     static_cast<int*>(ns.ptr), stream, 0, 0);
+}
+
+size_t fa_fwd_fp8_workspace_bytes(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1 || d != FP8_D) return 0;
+    if ((long long)B * H > 0x7fffffffLL || N > (1 << 30)) return 0;
+    return fp8_workspace_bytes((long long)B * H, N);
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B,
+                     int H, int N, int d, int causal, float scale, float descale_q,
+                     float descale_k, float descale_v, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+    if (!q8 || !k8 || !v8 || !o || !lse || !workspace) return FA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    for (float x : {scale, descale_q, descale_k, descale_v})
+        if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != FP8_D) return FA_ERR_UNSUPPORTED;
+    const long long BH = (long long)B * H;
+    if (BH > 0xffffLL || N > (1 << 30)) return FA_ERR_UNSUPPORTED;   // grid.y of the V^T pass
+    if (((long long)N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS * BH > (1LL << 30))
+        return FA_ERR_UNSUPPORTED;
+    if (workspace_bytes < fp8_workspace_bytes(BH, N)) return FA_ERR_INVALID_ARG;
+    if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(o, 16) ||
+        !aligned(lse, 4) || !aligned(workspace, 256))
+        return FA_ERR_MISALIGNED;
+    int dev = -1, sm_count = 0;
+    const fa_status ds = static_cast<fa_status>(fa_internal::current_device(&dev, &sm_count));
+    if (ds != FA_OK) return ds;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int* sched = static_cast<int*>(workspace);
+    uint8_t* vt = static_cast<uint8_t*>(workspace) + FA_DYNAMIC_WORKSPACE_BYTES;
+    const long long npad = fp8_npad(N);
+    CUtensorMap mq, mk, mv;
+    if (encode_map_e4m3(&mq, q8, FP8_D, N, H, B, fa::BM) != FA_OK ||
+        encode_map_e4m3(&mk, k8, FP8_D, N, H, B, fa::BN) != FA_OK ||
+        encode_map_e4m3(&mv, vt, npad, FP8_D, H, B, FP8_D) != FA_OK)
+        return FA_ERR_UNSUPPORTED;
+    transpose_v_e4m3<FP8_D><<<dim3(unsigned(npad / 64), unsigned(BH)), 256, 0, s>>>(
+        static_cast<const uint8_t*>(v8), vt, N, npad);
+    const float scale_log2 = scale * descale_q * descale_k * 1.4426950408889634f;
+    const Strides3 ost{(long long)H * N * FP8_D, (long long)N * FP8_D, (long long)FP8_D};
+    return launch_kernel<FP8_D, FP8_NS, true>(mq, mk, mv, o, lse, B, H, N, ost, causal, scale_log2,
+                                              descale_v, sched, s, dev, 4000ull * 1000000ull, 0);
 }
 
 fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -207,6 +207,42 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
                         int num_splits, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_fwd_fp8_workspace_bytes -- device workspace fa_fwd_fp8 needs: 256 bytes
+ * of work counter and the transposed V (B*H*d*Npad bytes, Npad = N rounded
+ * up to a multiple of 128).  Returns 0 for sizes fa_fwd_fp8 would reject.
+ */
+size_t fa_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * fa_fwd_fp8 -- exact attention forward over FP8 E4M3 inputs on the FP8 tensor
+ * cores (page "FlashAttention: The GPU Memory Hack That Changed Everything",
+ * "FlashAttention-3: Hopper Architecture": attention run in FP8 precision).
+ *
+ *  q8, k8, v8 : E4M3 codes [B][H][N][d], contiguous, d = 128; the values are
+ *               code * descale_q (resp. _k, _v), one scale per tensor.
+ *  o          : bf16 [B][H][N][d];  lse : fp32 [B][H][N], natural-log units
+ *               of scale * (descale_q q8) . (descale_k k8).
+ *  workspace  : device memory owned by the caller, 256-byte aligned, at least
+ *               fa_fwd_fp8_workspace_bytes(...) bytes; not shared by calls
+ *               that may run at the same time.
+ * S = Q K^T is formed exactly from the codes in fp32; P is rounded to E4M3
+ * (relative error up to 2^-4, values below 2^-6 on the E4M3 subnormal grid)
+ * before the P V product, while the row sum uses the unrounded fp32 P.  The
+ * work schedule is the one of fa_fwd_dynamic; a first pass writes V^T into
+ * the workspace so both tensor-core operands are K-major.
+ * Errors: FA_ERR_INVALID_ARG (NULL pointers, sizes < 1, bad causal flag, scale
+ * or descale not finite and > 0, workspace too small), FA_ERR_UNSUPPORTED
+ * (d != 128, B*H > 65535, sizes beyond the limits of fa_fwd, device not
+ * sm_100), FA_ERR_MISALIGNED (inputs or o not 16-byte aligned, lse not
+ * 4-byte aligned, workspace not 256-byte aligned), FA_ERR_NO_DEVICE,
+ * FA_ERR_LAUNCH.
+ */
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B,
+                     int H, int N, int d, int causal, float scale, float descale_q,
+                     float descale_k, float descale_v, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/*
  * fa_bwd_workspace_bytes -- device workspace fa_bwd needs for these sizes:
  * an fp32 dQ accumulator [B][H][Npad][d] and two fp32 per-row vectors
  * [B][H][Npad], Npad = N rounded up to a multiple of 128.  Returns 0 for

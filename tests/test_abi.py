@@ -23,7 +23,7 @@ def built_library():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_exports():
@@ -181,3 +181,29 @@ def test_bwd_argument_validation_and_workspace_size():
     assert fa.bwd_workspace_bytes(2, 3, 1000, 128) == 6 * 1024 * 128 * 4 + 2 * 6 * 1024 * 4
     assert fa.bwd_workspace_bytes(2, 3, 1000, 96) == 0
     assert fa.bwd_workspace_bytes(0, 3, 1000, 64) == 0
+
+
+def test_fp8_argument_validation_and_workspace_size():
+    W = 1 << 22
+    ok = [P, P, P, P, P, 2, 3, 1000, 128, 1, 0.1, 0.01, 0.02, 0.03, W, 1 << 30, 0]
+    assert fa.fa_fwd_fp8_raw(*ok) == fa.FA_ERR_NO_DEVICE                     # valid: stops at the device query
+    for i in (0, 1, 2, 3, 4, 14):                                             # NULL pointer or workspace
+        a = list(ok); a[i] = 0
+        assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_INVALID_ARG
+    for i in (10, 11, 12, 13):                                                # scale / descales
+        for bad in (0.0, -1.0, float("nan"), float("inf")):
+            a = list(ok); a[i] = bad
+            assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok); a[8] = 64
+    assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_UNSUPPORTED                    # d = 64
+    a = list(ok); a[5] = 300; a[6] = 300
+    assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_UNSUPPORTED                    # B*H > 65535
+    a = list(ok); a[15] = fa.fp8_workspace_bytes(2, 3, 1000, 128) - 1
+    assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_INVALID_ARG                    # workspace too small
+    a = list(ok); a[1] = P + 8
+    assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_MISALIGNED
+    a = list(ok); a[14] = W + 16
+    assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_MISALIGNED
+    # workspace: 256-byte work counter + V^T (B*H*d*Npad bytes, Npad = N rounded up to 128)
+    assert fa.fp8_workspace_bytes(2, 3, 1000, 128) == 256 + 6 * 128 * 1024
+    assert fa.fp8_workspace_bytes(2, 3, 1000, 64) == 0
