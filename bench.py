@@ -47,6 +47,7 @@ METRIC = "attention fwd TFLOP/s and % of B200 dense BF16 peak (1 GPU)"
 UNIT = "TFLOP/s"
 WORKLOAD_INDEX = 4          # long-context causal: B=2, H=32, N=8192, d=128
 KERNEL_SOURCE = os.path.join(ROOT, "exact_attention_122_b200", "csrc", "fa_fwd_sm100.cu")
+BWD_KERNEL_SOURCE = os.path.join(ROOT, "exact_attention_122_b200", "csrc", "fa_bwd_sm100.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAK_TFLOPS = 1590.0   # used only when the measured peaks file is absent
@@ -92,8 +93,8 @@ def sample_plan(w: synth.Workload, rows: int):
     return idx, 4.0 * keys * w.d
 
 
-def kernel_source_sha() -> str:
-    with open(KERNEL_SOURCE, "rb") as f:
+def kernel_source_sha(path: str = KERNEL_SOURCE) -> str:
+    with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()
 
 
@@ -106,17 +107,28 @@ def load_peaks():
         return FALLBACK_PEAK_TFLOPS, 0.0, "fallback"
 
 
-def load_traffic(workload_name: str):
-    """Per-launch DRAM bytes from the committed ncu summary, only while the
-    kernel source still matches the one that was profiled."""
+def load_traffic(workload_name: str, source: str = KERNEL_SOURCE):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summaries, only while that kernel's source file still matches the one
+    that was profiled.  The file holds {"entries": [...]}, each entry naming
+    its workload, its kernel source (relative to the repository) and that
+    source's sha256."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
-    if t.get("kernel_source_sha256") != kernel_source_sha() or t.get("workload") != workload_name:
-        return None
-    return t.get("bytes_per_launch")
+    entries = t.get("entries", [t]) if isinstance(t, dict) else []
+    rel = os.path.relpath(source, ROOT)
+    for e in entries:
+        if e.get("workload") != workload_name:
+            continue
+        if e.get("kernel_source", os.path.relpath(KERNEL_SOURCE, ROOT)) != rel:
+            continue
+        if e.get("kernel_source_sha256") != kernel_source_sha(source):
+            return None
+        return e.get("bytes_per_launch")
+    return None
 
 
 class ClockSampler:
@@ -541,7 +553,9 @@ def run_bwd(args):
                        "causal": w.causal, "flops_per_step": flops,
                        "l2": "inputs 537 MB > 126 MB L2; no flush"},
             "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s",
-                         "frac": value / peak, "traffic": None, "peak_source": peak_src,
+                         "frac": value / peak,
+                         "traffic": load_traffic(w.name + "_bwd", BWD_KERNEL_SOURCE),
+                         "traffic_kernel": "bwd_kernel", "peak_source": peak_src,
                          "kernel": "bwd_prep + bwd_kernel + bwd_dq_out (whole step)"},
             "gpu_launches": 3 * args.steps, "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
@@ -597,7 +611,8 @@ def run_fp8(args):
             "config": {"workload": w.name + "_fp8", "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                        "causal": w.causal, "l2": "inputs 268 MB > 126 MB L2; no flush"},
             "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s",
-                         "frac": value / peak, "traffic": None,
+                         "frac": value / peak, "traffic": load_traffic(w.name + "_fp8"),
+                         "traffic_kernel": "fa_fwd_kernel<128, 8, true>",
                          "peak_source": f"{peak_src} bf16 x 2 (nominal FP8/bf16 ratio)",
                          "kernel": "transpose_v_e4m3 + fa_fwd_kernel<128, 8, true> (whole step)"},
             "gpu_launches": 3 * args.steps, "clocks": clocks.summary()}

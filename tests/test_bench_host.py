@@ -56,6 +56,19 @@ def test_traffic_is_null_unless_kernel_matches(tmp_path, monkeypatch):
                              "workload": "long_context_causal", "bytes_per_launch": 123}))
     assert bench.load_traffic("long_context_causal") == 123
     assert bench.load_traffic("other") is None
+    # several entries, one per (workload, kernel source)
+    f.write_text(json.dumps({"entries": [
+        {"kernel_source": "exact_attention_122_b200/csrc/fa_fwd_sm100.cu",
+         "kernel_source_sha256": bench.kernel_source_sha(), "workload": "a", "bytes_per_launch": 1},
+        {"kernel_source": "exact_attention_122_b200/csrc/fa_bwd_sm100.cu",
+         "kernel_source_sha256": bench.kernel_source_sha(bench.BWD_KERNEL_SOURCE),
+         "workload": "a_bwd", "bytes_per_launch": 2},
+        {"kernel_source": "exact_attention_122_b200/csrc/fa_bwd_sm100.cu",
+         "kernel_source_sha256": "0" * 64, "workload": "b_bwd", "bytes_per_launch": 3}]}))
+    assert bench.load_traffic("a") == 1
+    assert bench.load_traffic("a_bwd", bench.BWD_KERNEL_SOURCE) == 2
+    assert bench.load_traffic("a_bwd") is None                     # wrong source for that entry
+    assert bench.load_traffic("b_bwd", bench.BWD_KERNEL_SOURCE) is None   # stale sha
 
 
 def _free_port():
