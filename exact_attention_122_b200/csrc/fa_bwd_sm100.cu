@@ -79,7 +79,6 @@ template <int D>
 struct Cfg {
     static constexpr int BQ = D == 128 ? 64 : 128;
     static constexpr bool DQ_T = D == 128;
-    static constexpr int NP = D == 128 ? 2 : 1;         // P buffers in TMEM
     static constexpr int KV_BYTES = BK * D * 2;
     static constexpr int KV_SLAB = BK * 128;             // 64 columns of a K/V tile
     static constexpr int QD_BYTES = BQ * D * 2;
@@ -100,7 +99,7 @@ struct Cfg {
     static constexpr int B_SDP_FULL = 1 + 2 * NS;
     static constexpr int B_SDP_FREE = 2 + 2 * NS;
     static constexpr int B_DS_READY = 3 + 2 * NS;        // [2]
-    static constexpr int B_P_FREE = 5 + 2 * NS;          // [2]
+    static constexpr int B_K_TMEM = 5 + 2 * NS;          // K copied into TMEM
     static constexpr int B_DS_FREE = 7 + 2 * NS;         // [2]
     static constexpr int B_DQ_FULL = 9 + 2 * NS;
     static constexpr int B_DQ_EMPTY = 10 + 2 * NS;
@@ -110,16 +109,22 @@ struct Cfg {
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem base, abort flag
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;
-    // TMEM columns
+    // TMEM columns.  P of block n (bf16, BQ/2 columns) lives in the first
+    // columns of the dQ region: it is written after the dQ warps have read
+    // dQ of block n-1, and the dQ MMA of block n overwrites it only after the
+    // dV MMA that reads it (MMAs from one thread run in issue order).  K is
+    // held in TMEM as the A operand of S^T = K Q^T (bf16, D/2 columns).
     static constexpr uint32_t TM_S = 0;
     static constexpr uint32_t TM_DP = BQ;
-    static constexpr uint32_t TM_P = 2 * BQ;                   // NP buffers of BQ/2 columns
-    static constexpr uint32_t TM_DQ = TM_P + NP * (BQ / 2);    // dQ^T: BQ cols; dQ: D cols
+    static constexpr uint32_t TM_DQ = 2 * BQ;                  // dQ^T: BQ cols; dQ: D cols
+    static constexpr uint32_t TM_P = TM_DQ;
     static constexpr uint32_t DQ_COLS = DQ_T ? BQ : D;
-    static constexpr uint32_t TM_DV = TM_DQ + DQ_COLS;
+    static constexpr uint32_t TM_K = TM_DQ + DQ_COLS;
+    static constexpr uint32_t TM_DV = TM_K + D / 2;
     static constexpr uint32_t TM_DK = TM_DV + D;
     static constexpr uint32_t TM_COLS = 512;
     static_assert(TM_DK + D <= TM_COLS, "TMEM budget");
+    static_assert(BQ / 2 <= DQ_COLS, "P fits in the dQ columns");
     static_assert(ALLOC <= 227 * 1024, "shared memory budget");
     static_assert(BYTES > 116 * 1024, "one CTA per SM keeps TMEM allocation uncontended");
     static_assert((BQ / 2) % 32 == 0, "compute warps take 32-column chunks");
@@ -377,11 +382,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         mbar_init(bar(C::B_SDP_FREE), COMPUTE_WARPS);
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(C::B_DS_READY + i), COMPUTE_WARPS);
-            mbar_init(bar(C::B_P_FREE + i), 1);
             mbar_init(bar(C::B_DS_FREE + i), 1);
         }
         mbar_init(bar(C::B_DQ_FULL), 1);
         mbar_init(bar(C::B_DQ_EMPTY), 4);
+        mbar_init(bar(C::B_K_TMEM), COMPUTE_WARPS);
         mbar_init(bar(C::B_ACC_FULL), 1);
         mbar_init(bar(C::B_DRAIN), 1);
         *abort_flag = 0;
@@ -447,14 +452,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             constexpr uint32_t ID_G = idesc_bf16(128, D, true);            // dV, dK
             constexpr uint32_t ID_Q = C::DQ_T ? idesc_bf16(128, BQ, true, true)   // dQ^T
                                               : idesc_bf16(128, D, true, true);   // dQ
-            const uint64_t dK_kmaj = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
             const uint64_t dV_kmaj = sdesc_sw128(sbase + C::OFF_V, 16, 1024);
             const uint64_t dK_mn = sdesc_sw128(sbase + C::OFF_K, C::KV_SLAB, 1024);
-            bool ok = wait_phase(bar(C::B_KV_FULL), 0, wd, ROLE_MMA, blk_id);
+            bool ok = wait_phase(bar(C::B_KV_FULL), 0, wd, ROLE_MMA, blk_id) &&
+                      wait_phase(bar(C::B_K_TMEM), 0, wd, ROLE_MMA, blk_id);
             tc_fence_after();
 
             auto grads = [&](int m) -> bool {
-                const int s = m % NS, pb = m % C::NP, db = m % 2;
+                const int s = m % NS, db = m % 2;
                 if (!wait_phase(bar(C::B_DS_READY + db), (m / 2) & 1, wd, ROLE_MMA, blk_id))
                     return false;
                 tc_fence_after();
@@ -466,10 +471,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 const uint64_t do_mn = sdesc_sw128(sdo, C::QD_SLAB, 1024);
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    mma_ts(tmem + C::TM_DV, tmem + C::TM_P + pb * (BQ / 2) + kk * 8,
+                    mma_ts(tmem + C::TM_DV, tmem + C::TM_P + kk * 8,
                            desc_add(do_mn, uint32_t((kk * 2048) >> 4)), ID_G,
                            (m > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar(C::B_P_FREE + pb));
                 // dK += dS^T Q: A = dS K-major (keys x queries), B = Q MN-major.
                 const uint64_t ds_kmaj = sdesc_sw128(sds, 16, 1024);
                 const uint64_t q_mn = sdesc_sw128(sq, C::QD_SLAB, 1024);
@@ -515,12 +519,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 const uint32_t sdo = sbase + C::OFF_DO + s * C::QD_BYTES;
                 const uint64_t q_kmaj = sdesc_sw128(sq, 16, 1024);
                 const uint64_t do_kmaj = sdesc_sw128(sdo, 16, 1024);
-                // S^T = K Q^T and dP^T = V dO^T: M = 128 keys, N = BQ queries, K = d.
+                // S^T = K Q^T (A = K from TMEM, 8 columns per 16 d) and
+                // dP^T = V dO^T (A = V from SMEM): M = 128 keys, N = BQ queries, K = d.
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t oa = uint32_t(((kk / 4) * C::KV_SLAB + (kk % 4) * 32) >> 4);
                     const uint32_t ob = uint32_t(((kk / 4) * C::QD_SLAB + (kk % 4) * 32) >> 4);
-                    mma_ss(tmem + C::TM_S, desc_add(dK_kmaj, oa), desc_add(q_kmaj, ob), ID_S,
+                    mma_ts(tmem + C::TM_S, tmem + C::TM_K + kk * 8, desc_add(q_kmaj, ob), ID_S,
                            kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
@@ -603,9 +607,31 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const int key = k0 + r;
         const uint32_t lane_base = uint32_t(32 * qw) << 16;
         const float cs = scale * LOG2E;
-        bool ok = true;
+        bool ok = warp_wait(bar(C::B_KV_FULL), 0, wd, ROLE_COMPUTE, blk_id);
+        if (ok) {
+            // K row r, d columns half*64 .. half*64+63 (one 128-byte swizzled
+            // slab row) -> TMEM columns TM_K + half*32 .. +31 as bf16 pairs.
+            uint32_t kr[32];
+            const uint32_t krow = sbase + C::OFF_K + half * C::KV_SLAB + (r / 8) * 1024 +
+                                  (r % 8) * 128;
+            if (half < D / 64) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t a = krow + uint32_t((c ^ (r % 8)) * 16);
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(kr[4 * c]), "=r"(kr[4 * c + 1]), "=r"(kr[4 * c + 2]),
+                                   "=r"(kr[4 * c + 3])
+                                 : "r"(a));
+                }
+                tmem_st32(tmem + lane_base + C::TM_K + half * 32, kr);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_K_TMEM));
+        }
         for (int n = 0; ok && n < nsteps; ++n) {
-            const int s = n % NS, pb = n % C::NP, db = n % 2;
+            const int s = n % NS, db = n % 2;
             const int q0 = (qb_first + n) * BQ;
             // QD_FULL: the LSE2 / D vectors of this block (bulk copies) have
             // landed; SDP_FULL: S^T and dP^T are in TMEM.
@@ -639,10 +665,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     p_ds_chunk<false>(sv, dpv, vl + col0, vd + col0, cs, q0 + col0, key, N, causal,
                                       pu, du);
                 if (c == 0) {
-                    // P buffer pb is free once dV of step n - NP has run; dS
-                    // buffer db once dK and dQ of step n - 2 have.
-                    if (n >= C::NP && !warp_wait(bar(C::B_P_FREE + pb), ((n / C::NP) - 1) & 1, wd,
-                                                 ROLE_COMPUTE, blk_id)) {
+                    // The P columns (dQ region) are free once the dQ warps have
+                    // read dQ of step n - 1; dS buffer db once dK and dQ of
+                    // step n - 2 have run.
+                    if (n >= 1 && !warp_wait(bar(C::B_DQ_EMPTY), (n - 1) & 1, wd, ROLE_COMPUTE,
+                                             blk_id)) {
                         ok = false;
                         break;
                     }
@@ -653,7 +680,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     }
                     tc_fence_after();
                 }
-                tmem_st16(tmem + lane_base + C::TM_P + pb * (BQ / 2) + col0 / 2, pu);
+                tmem_st16(tmem + lane_base + C::TM_P + col0 / 2, pu);
                 // dS row r, queries col0..col0+31, in the 128-byte-swizzled
                 // layout (16-byte chunk index XOR row % 8 inside 1 KiB atoms).
                 const uint32_t row_base = sds + (col0 / 64) * C::DS_SLAB + (r / 8) * 1024 +
