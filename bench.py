@@ -48,6 +48,7 @@ UNIT = "TFLOP/s"
 WORKLOAD_INDEX = 4          # long-context causal: B=2, H=32, N=8192, d=128
 KERNEL_SOURCE = os.path.join(ROOT, "exact_attention_122_b200", "csrc", "fa_fwd_sm100.cu")
 BWD_KERNEL_SOURCE = os.path.join(ROOT, "exact_attention_122_b200", "csrc", "fa_bwd_sm100.cu")
+DECODE_KERNEL_SOURCE = os.path.join(ROOT, "exact_attention_122_b200", "csrc", "fa_decode_sm100.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAK_TFLOPS = 1590.0   # used only when the measured peaks file is absent
@@ -493,7 +494,8 @@ def run_decode(args):
                        "causal": w.causal,
                        "l2": f"K+V {w.kv_bytes / 1e9:.1f} GB > 126 MB L2; no flush"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                         "frac": gbs / peak, "traffic": None, "peak_source": src,
+                         "frac": gbs / peak, "traffic": load_traffic(w.name, DECODE_KERNEL_SOURCE),
+                         "traffic_kernel": "decode_split_kernel", "peak_source": src,
                          "kernel": "decode_split_kernel + decode_merge_kernel"},
             "gpu_launches": 2 * args.steps, "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
