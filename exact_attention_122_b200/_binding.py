@@ -16,7 +16,8 @@ FA_ERR_NO_DEVICE = 6
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_dynamic_noalloc",
                     "fa_fwd_decode_workspace_bytes", "fa_fwd_decode", "fa_bwd_workspace_bytes",
-                    "fa_bwd", "fa_fwd_fp8_workspace_bytes", "fa_fwd_fp8", "fa_fwd_debug",
+                    "fa_bwd", "fa_bwd_debug", "fa_fwd_fp8_workspace_bytes", "fa_fwd_fp8",
+                    "fa_fwd_debug",
                     "fa_get_device_status", "fa_status_string", "fa_last_cuda_error", "fa_version")
 DECODE_MAX_QUERIES = 16                # FA_DECODE_MAX_QUERIES
 DECODE_MAX_SPLITS = 256                # FA_DECODE_MAX_SPLITS
@@ -62,6 +63,8 @@ def library() -> ctypes.CDLL:
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp,
                            ctypes.c_size_t, vp]
     lib.fa_bwd.restype = i
+    lib.fa_bwd_debug.argtypes = lib.fa_bwd.argtypes + [u, i]
+    lib.fa_bwd_debug.restype = i
     lib.fa_fwd_fp8_workspace_bytes.argtypes = [i, i, i, i]
     lib.fa_fwd_fp8_workspace_bytes.restype = ctypes.c_size_t
     lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, vp, ctypes.c_size_t,
@@ -193,6 +196,16 @@ def fa_bwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_
     """Direct call of fa_bwd; returns the fa_status code."""
     return library().fa_bwd(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr,
                             B, H, N, d, causal, scale, ws_ptr, ws_bytes, stream_ptr)
+
+
+def fa_bwd_debug_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr: int,
+                     dq_ptr: int, dk_ptr: int, dv_ptr: int, B: int, H: int, N: int, d: int,
+                     causal: int, scale: float, ws_ptr: int, ws_bytes: int, stream_ptr: int,
+                     watchdog_ms: int, inject: int) -> int:
+    """Direct call of fa_bwd_debug; returns the fa_status code."""
+    return library().fa_bwd_debug(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr,
+                                  dv_ptr, B, H, N, d, causal, scale, ws_ptr, ws_bytes, stream_ptr,
+                                  watchdog_ms, inject)
 
 
 def fa_bwd(q, k, v, out, lse, dout, causal: bool = False, scale: float | None = None,

@@ -340,7 +340,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
            const float* __restrict__ nlse2, const float* __restrict__ ndvec,
            float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
            __nv_bfloat16* __restrict__ dv, int BH, int H, int N, int Npad, int causal,
-           float scale, int hg, unsigned long long watchdog_ns) {
+           float scale, int hg, unsigned long long watchdog_ns, int inject) {
     using C = Cfg<D>;
     constexpr int BQ = C::BQ;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -417,11 +417,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                             bar(C::B_KV_FULL));
             }
             int issued = 0;
+            // Host-chosen fault injection (inject = 1): CTA 0 never issues its
+            // first Q / dO block, so the waits on it can only end by the watchdog.
+            const bool skip0 = inject == 1 && blockIdx.x == 0;
             for (int n = 0; n < nsteps; ++n) {
                 const int s = n % NS;
                 if (n >= NS && !wait_phase(bar(C::B_QD_EMPTY + s), ((n / NS) - 1) & 1, wd,
                                            ROLE_PRODUCER, blk_id))
                     break;
+                ++issued;
+                if (skip0 && n == 0) continue;
                 const int q0 = (qb_first + n) * BQ;
                 const uint32_t full = bar(C::B_QD_FULL + s);
                 mbar_arrive_expect_tx(full, 2 * C::QD_BYTES + C::VEC_BYTES);
@@ -436,12 +441,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 bulk_load(sbase + C::OFF_VEC + s * C::VEC_BYTES, nlse2 + vrow, BQ * 4, full);
                 bulk_load(sbase + C::OFF_VEC + s * C::VEC_BYTES + BQ * 4, ndvec + vrow, BQ * 4,
                           full);
-                ++issued;
             }
             // Drain: every copy this thread issued has landed before exit.
             wait_drain(bar(C::B_KV_FULL), 0, watchdog_ns);
             for (int n = (issued > NS ? issued - NS : 0); n < issued; ++n)
-                wait_drain(bar(C::B_QD_FULL + n % NS), (n / NS) & 1, watchdog_ns);
+                if (!(skip0 && n == 0))
+                    wait_drain(bar(C::B_QD_FULL + n % NS), (n / NS) & 1, watchdog_ns);
         }
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------------
@@ -769,7 +774,7 @@ template <int D>
 fa_status launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int causal,
                  float scale, unsigned char* ws, cudaStream_t stream, int dev,
-                 unsigned long long wd_ns) {
+                 unsigned long long wd_ns, int inject) {
     using C = Cfg<D>;
     const long long BH = (long long)B * H;
     const long long np = npad_of(N);
@@ -811,7 +816,8 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
     hg = hg < 1 ? 1 : (hg > BH ? BH : hg);
     bwd_kernel<D><<<unsigned(nkb * BH), NUM_THREADS, C::ALLOC, stream>>>(
         mq, mk, mv, mdo, nlse2, ndvec, dq_acc, static_cast<__nv_bfloat16*>(dk),
-        static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, int(hg), wd_ns);
+        static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, int(hg), wd_ns,
+        inject);
     const long long out_threads = BH * N * (D / 8);
     bwd_dq_out<D><<<unsigned((out_threads + 255) / 256), 256, 0, stream>>>(
         dq_acc, static_cast<__nv_bfloat16*>(dq), BH, N, int(np), scale);
@@ -844,15 +850,17 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
     return bwd::ws_layout((long long)B * H, N, d).total;
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+static fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                          int H, int N, int d, int causal, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream, unsigned watchdog_ms, int inject) {
     using bwd::aligned;
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
         return FA_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (inject != 0 && inject != 1) return FA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     const long long BH = (long long)B * H;
     if (BH > 0x7fffffffLL || N > (1 << 30)) return FA_ERR_UNSUPPORTED;
@@ -867,14 +875,29 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     int dev = -1, sm_count = 0;
     const int ds = fa_internal::current_device(&dev, &sm_count);
     if (ds != FA_OK) return static_cast<fa_status>(ds);
-    const unsigned long long wd_ns = 4000ull * 1000000ull;
+    const unsigned long long wd_ns = (watchdog_ms ? watchdog_ms : 4000u) * 1000000ull;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     if (d == 64)
         return bwd::launch<64>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, ws, s,
-                                  dev, wd_ns);
-    return bwd::launch<128>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, ws, s,
-                               dev, wd_ns);
+                               dev, wd_ns, inject);
+    return bwd::launch<128>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, ws, s, dev,
+                            wd_ns, inject);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace,
+                    workspace_bytes, stream, 0, 0);
+}
+
+fa_status fa_bwd_debug(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int H, int N, int d, int causal, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream, unsigned watchdog_ms, int inject) {
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace,
+                    workspace_bytes, stream, watchdog_ms, inject);
 }
 
 }  // extern "C"

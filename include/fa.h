@@ -285,6 +285,24 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int causal, float scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_bwd_debug -- fa_bwd with the kernel watchdog exposed, for tests.
+ *
+ *  watchdog_ms : every wait inside the backward kernel gives up after this
+ *                many milliseconds (0 = the default of 4000 ms), with the
+ *                same recovery as fa_fwd_debug (status word, bounded drain of
+ *                the CTA's own copies and MMAs, TMEM freed, context usable).
+ *  inject      : 0 = normal run.  1 = the producer of the first CTA never
+ *                issues its first Q / dO block, so the waits on it can only
+ *                end by the watchdog (host-chosen; no fault is involved).
+ * Other arguments and errors as fa_bwd.  dQ, dK, dV are undefined when the
+ * watchdog fires.
+ */
+fa_status fa_bwd_debug(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int H, int N, int d, int causal, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream, unsigned watchdog_ms, int inject);
+
+/*
  * fa_fwd_debug -- fa_fwd with the kernel watchdog exposed, for tests.
  *
  *  watchdog_ms : every wait inside the kernel gives up after this many

@@ -207,3 +207,10 @@ def test_fp8_argument_validation_and_workspace_size():
     # workspace: 256-byte work counter + V^T (B*H*d*Npad bytes, Npad = N rounded up to 128)
     assert fa.fp8_workspace_bytes(2, 3, 1000, 128) == 256 + 6 * 128 * 1024
     assert fa.fp8_workspace_bytes(2, 3, 1000, 64) == 0
+
+
+def test_bwd_debug_validates_inject():
+    W = 1 << 22
+    args = [P, P, P, P, P, P, P, P, P, 2, 3, 1000, 128, 1, 0.1, W, 1 << 30, 0]
+    assert fa.fa_bwd_debug_raw(*args, 100, 7) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_bwd_debug_raw(*args, 100, 1) == fa.FA_ERR_NO_DEVICE       # valid: stops at the device query

@@ -189,3 +189,28 @@ def test_bwd_argument_errors_on_device(fa):
     assert fa.fa_bwd_raw(*bad, ws.numel(), s) == fa.FA_ERR_MISALIGNED
     torch.cuda.synchronize()
     assert fa.device_status()[0] == fa.FA_OK
+
+
+def test_bwd_watchdog_reports_timeout_and_context_survives(fa):
+    """Host-chosen fault injection: CTA 0's producer never issues its first
+    Q / dO block.  The waits on it end by the watchdog (200 ms), the status
+    word reads FA_ERR_TIMEOUT, and the next call is correct."""
+    B, H, N, d = 1, 2, 512, 128
+    q, k, v = synth.draw_qkv(B, H, N, d, seed=71)
+    do = synth.draw_dout(B, H, N, d, seed=71)
+    qd, kd, vd, dod = (t.to("cuda:0") for t in (q, k, v, do))
+    o, lse = fa.fa_fwd(qd, kd, vd, causal=True)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda:0")
+    s = torch.cuda.current_stream().cuda_stream
+    torch.cuda.synchronize()
+    assert fa.device_status()[0] == fa.FA_OK
+    st = fa.fa_bwd_debug_raw(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), o.data_ptr(),
+                             dod.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                             dv.data_ptr(), B, H, N, d, 1, 1 / math.sqrt(d), ws.data_ptr(),
+                             ws.numel(), s, 200, 1)
+    assert st == fa.FA_OK
+    st, word = fa.device_status(s)
+    assert st == fa.FA_ERR_TIMEOUT, (fa.status_string(st), hex(word))
+    assert fa.device_status(s)[0] == fa.FA_OK                      # read-and-clear
+    compare_all(fa, B, H, N, d, True, seed=71)                     # the context still works
