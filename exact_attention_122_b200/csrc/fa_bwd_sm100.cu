@@ -47,6 +47,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "fa.h"
 #include "fa_internal.h"
@@ -754,6 +755,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;             // current_device() accepts indices below this
+
 long long npad_of(int N) { return ((long long)N + BK - 1) / BK * BK; }
 
 struct WsLayout {
@@ -791,11 +794,15 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
         fa_internal::encode_bhnd_map(&mdo, dout, D, N, H, B, sb, sh, sn, C::BQ) != FA_OK)
         return FA_ERR_UNSUPPORTED;
 
-    // Per-device, idempotent and cheap; set on every call so a device switch
-    // between calls is covered.
-    (void)dev;
-    cudaError_t e = cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::ALLOC);
+    // The dynamic shared-memory limit is a per-device function attribute: set
+    // once per (instantiation, device).
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t attr_err[kMaxDevices];
+    std::call_once(once[dev], [&] {
+        attr_err[dev] = cudaFuncSetAttribute(bwd_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::ALLOC);
+    });
+    cudaError_t e = attr_err[dev];
     if (e != cudaSuccess) {
         fa_internal::set_last_cuda_error(int(e));
         return FA_ERR_LAUNCH;
