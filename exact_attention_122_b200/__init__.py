@@ -15,3 +15,4 @@ from ._binding import (  # noqa: F401
     fa_fwd_debug_raw, device_status, bwd_workspace_bytes, fa_bwd, fa_bwd_raw, fa_bwd_debug_raw,
     fp8_workspace_bytes, fa_fwd_fp8, fa_fwd_fp8_raw,
 )
+from .autograd import attention  # noqa: F401,E402

@@ -214,3 +214,21 @@ def test_bwd_watchdog_reports_timeout_and_context_survives(fa):
     assert st == fa.FA_ERR_TIMEOUT, (fa.status_string(st), hex(word))
     assert fa.device_status(s)[0] == fa.FA_OK                      # read-and-clear
     compare_all(fa, B, H, N, d, True, seed=71)                     # the context still works
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_autograd_attention_matches_oracle(fa, causal):
+    """exact_attention_122_b200.attention under torch.autograd: loss = sum(O * dO)
+    gives dL/dq, dL/dk, dL/dv = the oracle's gradients for upstream dO."""
+    B, H, N, d = 2, 2, 333, 64
+    q, k, v = synth.draw_qkv(B, H, N, d, seed=73)
+    do = synth.draw_dout(B, H, N, d, seed=73)
+    qd, kd, vd = (t.to("cuda:0").requires_grad_(True) for t in (q, k, v))
+    o = fa.attention(qd, kd, vd, causal=causal)
+    (o.float() * do.to("cuda:0").float()).sum().backward()
+    dQ, dK, dV, _ = oracle.attention_bwd_fp64(q, k, v, do, causal=causal, scale=1 / math.sqrt(d))
+    check_grad(qd.grad, dQ, "autograd dQ")
+    check_grad(kd.grad, dK, "autograd dK")
+    check_grad(vd.grad, dV, "autograd dV")
+    O_ref, _ = oracle.attention_fp64(q, k, v, causal=causal, scale=1 / math.sqrt(d))
+    assert float(np.abs(o.detach().float().cpu().numpy() - O_ref).max()) <= 2e-2
