@@ -495,8 +495,8 @@ def run_decode(args):
                        "l2": f"K+V {w.kv_bytes / 1e9:.1f} GB > 126 MB L2; no flush"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": load_traffic(w.name, DECODE_KERNEL_SOURCE),
-                         "traffic_kernel": "decode_split_kernel", "peak_source": src,
-                         "kernel": "decode_split_kernel + decode_merge_kernel"},
+                         "traffic_kernel": "decode_mma_kernel", "peak_source": src,
+                         "kernel": "decode_mma_kernel + decode_merge_kernel"},
             "gpu_launches": 2 * args.steps, "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
     return 0

@@ -186,8 +186,9 @@ size_t fa_fwd_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d, int nu
  * each range keeps the online-softmax running state of the page "Flash
  * attention optimization" ("The fix: tile the computation ..."), and a
  * second kernel merges the ranges with that page's rescale-and-merge rule.
- * This shape is bound by reading K and V once from device memory, so it
- * runs on the CUDA cores.  P stays in fp32 here (no bf16 rounding of P).
+ * This shape is bound by reading K and V once from device memory.  The
+ * queries are padded to 16 rows for warp-level bf16 tensor-core MMAs, and P
+ * is rounded to bf16 before the P V product, as in fa_fwd.
  *
  *  Nq          : 1 .. FA_DECODE_MAX_QUERIES.
  *  Nk          : >= 1 (>= Nq when causal), <= 2^30;  B*H <= 65535.

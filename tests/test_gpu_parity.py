@@ -359,6 +359,9 @@ DECODE_CASES = [
     (2, 4, 1, 4096, 128, False, 0), (2, 4, 1, 4097, 64, True, 0), (1, 8, 16, 3000, 128, True, 0),
     (3, 2, 7, 130, 64, True, 3), (1, 2, 5, 5, 128, True, 0), (1, 1, 1, 1, 64, False, 0),
     (2, 3, 3, 1000, 128, True, 1), (2, 3, 3, 1000, 128, False, 9), (1, 4, 12, 20000, 128, True, 0),
+    # tensor-core kernel (5 <= Nq <= 16): ragged key tiles, few keys, explicit splits
+    (2, 3, 9, 777, 64, False, 0), (1, 2, 16, 33, 64, True, 2), (1, 3, 6, 4096, 128, False, 5),
+    (1, 2, 16, 1, 128, False, 0), (2, 2, 8, 8, 128, True, 0), (1, 2, 13, 2049, 128, True, 0),
 ]
 
 
