@@ -16,7 +16,8 @@ FA_ERR_NO_DEVICE = 6
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_dynamic_noalloc",
                     "fa_fwd_decode_workspace_bytes", "fa_fwd_decode", "fa_bwd_workspace_bytes",
-                    "fa_bwd", "fa_bwd_debug", "fa_fwd_fp8_workspace_bytes", "fa_fwd_fp8",
+                    "fa_bwd", "fa_bwd_strided", "fa_bwd_debug", "fa_fwd_fp8_workspace_bytes",
+                    "fa_fwd_fp8",
                     "fa_fwd_debug",
                     "fa_get_device_status", "fa_status_string", "fa_last_cuda_error", "fa_version")
 DECODE_MAX_QUERIES = 16                # FA_DECODE_MAX_QUERIES
@@ -63,6 +64,9 @@ def library() -> ctypes.CDLL:
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp,
                            ctypes.c_size_t, vp]
     lib.fa_bwd.restype = i
+    lib.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
+                                   ctypes.POINTER(ctypes.c_longlong), i, f, vp, ctypes.c_size_t, vp]
+    lib.fa_bwd_strided.restype = i
     lib.fa_bwd_debug.argtypes = lib.fa_bwd.argtypes + [u, i]
     lib.fa_bwd_debug.restype = i
     lib.fa_fwd_fp8_workspace_bytes.argtypes = [i, i, i, i]
@@ -198,6 +202,17 @@ def fa_bwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_
                             B, H, N, d, causal, scale, ws_ptr, ws_bytes, stream_ptr)
 
 
+def fa_bwd_strided_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr: int,
+                       dq_ptr: int, dk_ptr: int, dv_ptr: int, B: int, H: int, N: int, d: int,
+                       strides, causal: int, scale: float, ws_ptr: int, ws_bytes: int,
+                       stream_ptr: int) -> int:
+    """Direct call of fa_bwd_strided (strides: 24 ints or None); returns the fa_status code."""
+    arr = None if strides is None else (ctypes.c_longlong * 24)(*strides)
+    return library().fa_bwd_strided(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr,
+                                    dv_ptr, B, H, N, d, arr, causal, scale, ws_ptr, ws_bytes,
+                                    stream_ptr)
+
+
 def fa_bwd_debug_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr: int,
                      dq_ptr: int, dk_ptr: int, dv_ptr: int, B: int, H: int, N: int, d: int,
                      causal: int, scale: float, ws_ptr: int, ws_bytes: int, stream_ptr: int,
@@ -210,15 +225,18 @@ def fa_bwd_debug_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int
 
 def fa_bwd(q, k, v, out, lse, dout, causal: bool = False, scale: float | None = None,
            dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """dQ, dK, dV of attention for contiguous bf16 CUDA tensors q, k, v, out,
-    dout (B, H, N, d) and the forward's fp32 lse (B, H, N).  ``workspace`` (at
-    least bwd_workspace_bytes(B, H, N, d) bytes of device memory) is allocated
-    with torch when not given."""
+    """dQ, dK, dV of attention for bf16 CUDA tensors q, k, v, out, dout
+    (B, H, N, d) and the forward's fp32 lse (B, H, N, contiguous).  The bf16
+    tensors may be strided views with a contiguous last dimension (strided
+    calls go through fa_bwd_strided); dq, dk, dv are allocated contiguous when
+    not given.  ``workspace`` (at least bwd_workspace_bytes(B, H, N, d) bytes
+    of device memory) is allocated with torch when not given."""
     import torch
 
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
-        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.is_contiguous()):
-            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 4 and t.stride(-1) == 1):
+            raise ValueError(f"{name} must be a bf16 CUDA tensor (B, H, N, d) with a contiguous "
+                             "last dimension")
     B, H, N, d = q.shape
     for t in (k, v, out, dout):
         if t.shape != q.shape:
@@ -228,18 +246,29 @@ def fa_bwd(q, k, v, out, lse, dout, causal: bool = False, scale: float | None = 
         raise ValueError("lse must be a contiguous fp32 CUDA tensor (B, H, N)")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.shape == q.shape and t.stride(-1) == 1):
+            raise ValueError(f"{name} must be a bf16 CUDA tensor shaped like q with a contiguous "
+                             "last dimension")
     need = bwd_workspace_bytes(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    tensors = (q, k, v, out, dout, dq, dk, dv)
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
-        st = fa_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
-                        lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
-                        1 if causal else 0, float(scale), workspace.data_ptr(),
-                        workspace.numel() * workspace.element_size(), s.cuda_stream)
+        args = [t.data_ptr() for t in tensors[:5]] + [lse.data_ptr()] + \
+               [t.data_ptr() for t in tensors[5:]]
+        ws = (workspace.data_ptr(), workspace.numel() * workspace.element_size())
+        if all(t.is_contiguous() for t in tensors):
+            st = fa_bwd_raw(*args, B, H, N, d, 1 if causal else 0, float(scale), *ws,
+                            s.cuda_stream)
+        else:
+            strides = [x for t in tensors for x in t.stride()[:3]]
+            st = fa_bwd_strided_raw(*args, B, H, N, d, strides, 1 if causal else 0, float(scale),
+                                    *ws, s.cuda_stream)
     if st != FA_OK:
         raise FaError(st, "fa_bwd")
     return dq, dk, dv

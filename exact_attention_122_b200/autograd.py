@@ -19,7 +19,9 @@ from . import _binding
 class _ExactAttention(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, causal: bool, scale: float):
-        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        # Views with a contiguous last dimension (e.g. BNHD transposed) go
+        # through the strided entry points as they are; others are copied.
+        q, k, v = (t if t.stride(-1) == 1 else t.contiguous() for t in (q, k, v))
         o, lse = _binding.fa_fwd(q, k, v, causal=causal, scale=scale)
         ctx.save_for_backward(q, k, v, o, lse)
         ctx.causal = causal
@@ -30,8 +32,8 @@ class _ExactAttention(torch.autograd.Function):
     @staticmethod
     def backward(ctx, do, _dlse):
         q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = _binding.fa_bwd(q, k, v, o, lse, do.contiguous(), causal=ctx.causal,
-                                     scale=ctx.scale)
+        do = do if do.stride(-1) == 1 else do.contiguous()
+        dq, dk, dv = _binding.fa_bwd(q, k, v, o, lse, do, causal=ctx.causal, scale=ctx.scale)
         return dq, dk, dv, None, None
 
 

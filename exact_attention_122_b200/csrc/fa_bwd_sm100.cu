@@ -131,6 +131,15 @@ struct Cfg {
     static_assert((BQ / 2) % 32 == 0, "compute warps take 32-column chunks");
 };
 
+// Element strides (batch, head, sequence) of one bf16 [B][H][N][d] operand;
+// the head dimension d is contiguous.
+struct St3 {
+    long long b, h, n;
+    __host__ __device__ long long row(long long bh, int H, long long r) const {
+        return (bh / H) * b + (bh % H) * h + r * n;
+    }
+};
+
 __device__ unsigned int g_bwd_status;   // 0 = fine; else (FA_ERR_TIMEOUT << 24) | role << 20 | block
 
 struct Watchdog {
@@ -226,8 +235,8 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict_
                                                 const float* __restrict__ lse,
                                                 float* __restrict__ nlse2,
                                                 float* __restrict__ ndvec,
-                                                float* __restrict__ dq_acc, long long BH, int N,
-                                                int Npad) {
+                                                float* __restrict__ dq_acc, long long BH, int H,
+                                                int N, int Npad, St3 so, St3 sdo) {
     constexpr int TPR = D / 8;                          // threads per row
     const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long row = t / TPR;                      // over BH * Npad
@@ -237,9 +246,8 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict_
     const int r = int(row - bh * Npad);
     float acc = 0.f;
     if (live && r < N) {
-        const long long e = ((bh * N + r) * D) + part * 8;
-        const uint4 a = *reinterpret_cast<const uint4*>(o + e);
-        const uint4 b = *reinterpret_cast<const uint4*>(dout + e);
+        const uint4 a = *reinterpret_cast<const uint4*>(o + so.row(bh, H, r) + part * 8);
+        const uint4 b = *reinterpret_cast<const uint4*>(dout + sdo.row(bh, H, r) + part * 8);
         const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
         const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
@@ -266,7 +274,7 @@ __global__ void __launch_bounds__(256) bwd_prep(const __nv_bfloat16* __restrict_
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dq_out(const float* __restrict__ dq_acc,
                                                   __nv_bfloat16* __restrict__ dq, long long BH,
-                                                  int N, int Npad, float scale) {
+                                                  int H, int N, int Npad, float scale, St3 sdq) {
     constexpr int TPR = D / 8;
     const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long row = t / TPR;                      // over BH * N
@@ -281,7 +289,7 @@ __global__ void __launch_bounds__(256) bwd_dq_out(const float* __restrict__ dq_a
     out.y = pack_bf16x2(scale * x.z, scale * x.w);
     out.z = pack_bf16x2(scale * y.x, scale * y.y);
     out.w = pack_bf16x2(scale * y.z, scale * y.w);
-    *reinterpret_cast<uint4*>(dq + row * D + part * 8) = out;
+    *reinterpret_cast<uint4*>(dq + sdq.row(bh, H, r) + part * 8) = out;
 }
 
 // P and dS for 32 query columns of one key row (this thread's TMEM lane):
@@ -341,7 +349,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
            const float* __restrict__ nlse2, const float* __restrict__ ndvec,
            float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
            __nv_bfloat16* __restrict__ dv, int BH, int H, int N, int Npad, int causal,
-           float scale, int hg, unsigned long long watchdog_ns, int inject) {
+           float scale, int hg, unsigned long long watchdog_ns, int inject, St3 sdk, St3 sdv) {
     using C = Cfg<D>;
     constexpr int BQ = C::BQ;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -717,7 +725,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             for (int which = 0; which < 2; ++which) {
                 const uint32_t tcol = (which == 0 ? C::TM_DV : C::TM_DK) + half * HC;
                 const float mul = which == 0 ? 1.f : scale;
-                __nv_bfloat16* dst = (which == 0 ? dv : dk) + ((long long)bh * N + key) * D + half * HC;
+                __nv_bfloat16* dst = (which == 0 ? dv + sdv.row(bh, H, key) : dk + sdk.row(bh, H, key)) +
+                                     half * HC;
 #pragma unroll
                 for (int c = 0; c < HC / 32; ++c) {
                     uint32_t x[32];
@@ -775,9 +784,9 @@ WsLayout ws_layout(long long BH, int N, int d) {
 
 template <int D>
 fa_status launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int causal,
-                 float scale, unsigned char* ws, cudaStream_t stream, int dev,
-                 unsigned long long wd_ns, int inject) {
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N,
+                 const St3 (&st)[8], int causal, float scale, unsigned char* ws,
+                 cudaStream_t stream, int dev, unsigned long long wd_ns, int inject) {
     using C = Cfg<D>;
     const long long BH = (long long)B * H;
     const long long np = npad_of(N);
@@ -786,12 +795,13 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
     float* nlse2 = reinterpret_cast<float*>(ws + wl.nlse2);
     float* ndvec = reinterpret_cast<float*>(ws + wl.ndvec);
 
-    const long long sb = (long long)H * N * D, sh = (long long)N * D, sn = D;
+    // Operand order of st: q, k, v, o, dout, dq, dk, dv.
     CUtensorMap mq, mk, mv, mdo;
-    if (fa_internal::encode_bhnd_map(&mq, q, D, N, H, B, sb, sh, sn, C::BQ) != FA_OK ||
-        fa_internal::encode_bhnd_map(&mk, k, D, N, H, B, sb, sh, sn, BK) != FA_OK ||
-        fa_internal::encode_bhnd_map(&mv, v, D, N, H, B, sb, sh, sn, BK) != FA_OK ||
-        fa_internal::encode_bhnd_map(&mdo, dout, D, N, H, B, sb, sh, sn, C::BQ) != FA_OK)
+    auto enc = [&](CUtensorMap* m, const void* p, const St3& x, int rows) {
+        return fa_internal::encode_bhnd_map(m, p, D, N, H, B, x.b, x.h, x.n, rows);
+    };
+    if (enc(&mq, q, st[0], C::BQ) != FA_OK || enc(&mk, k, st[1], BK) != FA_OK ||
+        enc(&mv, v, st[2], BK) != FA_OK || enc(&mdo, dout, st[4], C::BQ) != FA_OK)
         return FA_ERR_UNSUPPORTED;
 
     // The dynamic shared-memory limit is a per-device function attribute: set
@@ -811,7 +821,7 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
     const long long prep_threads = BH * np * (D / 8);
     bwd_prep<D><<<unsigned((prep_threads + 255) / 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, nlse2,
-        ndvec, dq_acc, BH, N, int(np));
+        ndvec, dq_acc, BH, H, N, int(np), st[3], st[4]);
     const long long nkb = (N + BK - 1) / BK;
     // Heads per group: about 48 MiB of per-head data (Q, dO, K, V in bf16 and
     // the fp32 dQ accumulator, 12 bytes per element of one tensor) so the
@@ -824,10 +834,10 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
     bwd_kernel<D><<<unsigned(nkb * BH), NUM_THREADS, C::ALLOC, stream>>>(
         mq, mk, mv, mdo, nlse2, ndvec, dq_acc, static_cast<__nv_bfloat16*>(dk),
         static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, int(hg), wd_ns,
-        inject);
+        inject, st[6], st[7]);
     const long long out_threads = BH * N * (D / 8);
     bwd_dq_out<D><<<unsigned((out_threads + 255) / 256), 256, 0, stream>>>(
-        dq_acc, static_cast<__nv_bfloat16*>(dq), BH, N, int(np), scale);
+        dq_acc, static_cast<__nv_bfloat16*>(dq), BH, H, N, int(np), scale, st[5]);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         fa_internal::set_last_cuda_error(int(e));
@@ -859,8 +869,9 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
 
 static fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
                           const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                          int H, int N, int d, int causal, float scale, void* workspace,
-                          size_t workspace_bytes, void* stream, unsigned watchdog_ms, int inject) {
+                          int H, int N, int d, const long long* strides24, int causal, float scale,
+                          void* workspace, size_t workspace_bytes, void* stream,
+                          unsigned watchdog_ms, int inject) {
     using bwd::aligned;
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
         return FA_ERR_INVALID_ARG;
@@ -878,6 +889,25 @@ static fa_status bwd_impl(const void* q, const void* k, const void* v, const voi
         !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
         !aligned(lse, 4) || !aligned(workspace, 256))
         return FA_ERR_MISALIGNED;
+    // Strides of q, k, v, o, dout, dq, dk, dv, each (batch, head, sequence) in
+    // elements; NULL means contiguous [B][H][N][d].  Same rules as the
+    // forward's: >= d, a multiple of 8 elements (16 bytes), below 2^39; the
+    // stride of a dimension of size 1 is never used.
+    bwd::St3 st[8];
+    for (int i = 0; i < 8; ++i) {
+        if (strides24)
+            st[i] = bwd::St3{strides24[3 * i], strides24[3 * i + 1], strides24[3 * i + 2]};
+        else
+            st[i] = bwd::St3{(long long)H * N * d, (long long)N * d, (long long)d};
+        if (B == 1) st[i].b = d;
+        if (H == 1) st[i].h = d;
+        if (N == 1) st[i].n = d;
+        for (long long x : {st[i].b, st[i].h, st[i].n}) {
+            if (x < d) return FA_ERR_INVALID_ARG;
+            if ((x * 2) % 16 != 0) return FA_ERR_MISALIGNED;
+            if (x * 2 >= (1LL << 40)) return FA_ERR_UNSUPPORTED;
+        }
+    }
 
     int dev = -1, sm_count = 0;
     const int ds = fa_internal::current_device(&dev, &sm_count);
@@ -886,25 +916,34 @@ static fa_status bwd_impl(const void* q, const void* k, const void* v, const voi
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     if (d == 64)
-        return bwd::launch<64>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, ws, s,
-                               dev, wd_ns, inject);
-    return bwd::launch<128>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, ws, s, dev,
-                            wd_ns, inject);
+        return bwd::launch<64>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, st, causal, scale, ws,
+                               s, dev, wd_ns, inject);
+    return bwd::launch<128>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, st, causal, scale, ws, s,
+                            dev, wd_ns, inject);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                  int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
-    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace,
-                    workspace_bytes, stream, 0, 0);
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, nullptr, causal, scale,
+                    workspace, workspace_bytes, stream, 0, 0);
+}
+
+fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, const long long* strides, int causal, float scale,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    if (!strides) return FA_ERR_INVALID_ARG;
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, strides, causal, scale,
+                    workspace, workspace_bytes, stream, 0, 0);
 }
 
 fa_status fa_bwd_debug(const void* q, const void* k, const void* v, const void* o,
                        const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                        int H, int N, int d, int causal, float scale, void* workspace,
                        size_t workspace_bytes, void* stream, unsigned watchdog_ms, int inject) {
-    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace,
-                    workspace_bytes, stream, watchdog_ms, inject);
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, nullptr, causal, scale,
+                    workspace, workspace_bytes, stream, watchdog_ms, inject);
 }
 
 }  // extern "C"

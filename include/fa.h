@@ -286,6 +286,25 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int causal, float scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_bwd_strided -- fa_bwd for strided operands, e.g. [B][N][H][d] tensors
+ * viewed as (B, H, N, d).
+ *
+ *  strides : 24 int64 values, element strides (batch, head, sequence) of q,
+ *            k, v, o, dout, dq, dk and dv in that order, with the rules of
+ *            fa_fwd_strided (>= d, a multiple of 8 elements, below 2^39, the
+ *            stride of a dimension of size 1 ignored).  The head dimension d
+ *            is always contiguous.  Rows of dq, dk and dv must not overlap
+ *            each other or any input.
+ *  lse     : contiguous float [B][H][N] as in fa_bwd.
+ * Other arguments, results and errors as fa_bwd; FA_ERR_INVALID_ARG also for
+ * a NULL `strides`, and the stride errors of fa_fwd_strided.
+ */
+fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, const long long* strides, int causal, float scale,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_bwd_debug -- fa_bwd with the kernel watchdog exposed, for tests.
  *
  *  watchdog_ms : every wait inside the backward kernel gives up after this

@@ -214,3 +214,19 @@ def test_bwd_debug_validates_inject():
     args = [P, P, P, P, P, P, P, P, P, 2, 3, 1000, 128, 1, 0.1, W, 1 << 30, 0]
     assert fa.fa_bwd_debug_raw(*args, 100, 7) == fa.FA_ERR_INVALID_ARG
     assert fa.fa_bwd_debug_raw(*args, 100, 1) == fa.FA_ERR_NO_DEVICE       # valid: stops at the device query
+
+
+def test_bwd_strided_argument_validation():
+    W = 1 << 22
+    B, H, N, d = 2, 3, 8, 64
+    st = [H * N * d, N * d, d] * 8
+    base = [P, P, P, P, P, P, P, P, P, B, H, N, d]
+    tail = [1, 0.1, W, 1 << 30, 0]
+    assert fa.fa_bwd_strided_raw(*base, st, *tail) == fa.FA_ERR_NO_DEVICE   # valid
+    assert fa.fa_bwd_strided_raw(*base, None, *tail) == fa.FA_ERR_INVALID_ARG
+    bad = list(st); bad[17] = 32                                         # dq seq stride < d
+    assert fa.fa_bwd_strided_raw(*base, bad, *tail) == fa.FA_ERR_INVALID_ARG
+    bad = list(st); bad[22] = 130                                        # dv head stride not 8-aligned
+    assert fa.fa_bwd_strided_raw(*base, bad, *tail) == fa.FA_ERR_MISALIGNED
+    bad = list(st); bad[12] = 1 << 40                                    # dout batch stride too large
+    assert fa.fa_bwd_strided_raw(*base, bad, *tail) == fa.FA_ERR_UNSUPPORTED

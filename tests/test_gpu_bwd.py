@@ -232,3 +232,33 @@ def test_autograd_attention_matches_oracle(fa, causal):
     check_grad(vd.grad, dV, "autograd dV")
     O_ref, _ = oracle.attention_fp64(q, k, v, causal=causal, scale=1 / math.sqrt(d))
     assert float(np.abs(o.detach().float().cpu().numpy() - O_ref).max()) <= 2e-2
+
+
+def _bnhd(t):
+    """A (B, H, N, d) view of a [B][N][H][d] tensor holding the same values."""
+    return t.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+
+
+@pytest.mark.parametrize("d,N,causal", [(64, 300, True), (128, 513, False), (128, 1024, True)])
+def test_bwd_strided_views_match_contiguous(fa, d, N, causal):
+    """BNHD views of every operand (inputs and outputs) give the same dK and
+    dV bits as the contiguous call and dQ equal up to the order of its atomic
+    fp32 additions; both match the oracle."""
+    B, H = 2, 3
+    q, k, v = synth.draw_qkv(B, H, N, d, seed=77 + N)
+    do = synth.draw_dout(B, H, N, d, seed=77 + N)
+    qd, kd, vd, dod = (t.to("cuda:0") for t in (q, k, v, do))
+    o, lse = fa.fa_fwd(qd, kd, vd, causal=causal)
+    dq0, dk0, dv0 = fa.fa_bwd(qd, kd, vd, o, lse, dod, causal=causal)
+    qs, ks, vs, os_, dos = (_bnhd(t) for t in (qd, kd, vd, o, dod))
+    outs = [_bnhd(torch.empty_like(qd)) for _ in range(3)]
+    assert not qs.is_contiguous() and not outs[0].is_contiguous()
+    dq1, dk1, dv1 = fa.fa_bwd(qs, ks, vs, os_, lse, dos, causal=causal, dq=outs[0], dk=outs[1],
+                              dv=outs[2])
+    torch.cuda.synchronize()
+    assert torch.equal(dk1, dk0) and torch.equal(dv1, dv0)
+    assert float((dq1.float() - dq0.float()).abs().max()) <= 1e-2 * float(dq0.float().abs().max())
+    dQ, dK, dV, _ = oracle.attention_bwd_fp64(q, k, v, do, causal=causal, scale=1 / math.sqrt(d))
+    check_grad(dq1, dQ, "strided dQ")
+    check_grad(dk1, dK, "strided dK")
+    check_grad(dv1, dV, "strided dV")
