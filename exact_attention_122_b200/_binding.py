@@ -290,7 +290,7 @@ def fa_fwd_fp8(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float,
                causal: bool = False, scale: float | None = None, out=None, lse=None,
                workspace=None, stream=None):
     """O (bf16), LSE of attention over FP8 E4M3 inputs: q8, k8, v8 contiguous
-    CUDA tensors (B, H, N, 128) of dtype uint8 or torch.float8_e4m3fn holding
+    CUDA tensors (B, H, N, d), d in {64, 128}, of dtype uint8 or torch.float8_e4m3fn holding
     the codes; the values are code * descale_x.  ``workspace`` (at least
     fp8_workspace_bytes(B, H, N, d) bytes) is allocated with torch when not
     given."""

@@ -105,7 +105,10 @@ struct Layout {
     static constexpr int Q_BYTES = BM * D * EB;      // one sub-tile of Q
     static constexpr int KV_BYTES = BN * D * EB;     // one K or V tile
     static constexpr int HALF_BYTES = BM * 128;      // one 128-byte-wide slab (16 KiB)
-    static constexpr int SLABS = D * EB / 128;       // slabs per Q / K tile
+    // FP8 at d = 64: a Q / K row is 64 bytes, held in 64-byte-swizzled tiles
+    // (one slab); every other case uses 128-byte rows.
+    static constexpr bool SW64 = F8 && D == 64;
+    static constexpr int SLABS = SW64 ? 1 : D * EB / 128;   // slabs per Q / K tile
     static constexpr int SLAB_ELEMS = 128 / EB;      // elements per slab row
     static constexpr int QK_STEPS = D * EB / 32;     // 32-byte K steps of S = Q K^T
     static constexpr int OFF_Q = 0;
@@ -513,9 +516,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // Descriptors, built once: Q sub-tiles and ring stages (K-major
             // view for K, MN-major view for V: leading byte offset = the
             // 16 KiB between d slabs, stride byte offset = 8 rows x 128 B).
-            const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
-            const uint64_t dq1 = sdesc_sw128(sQ + L::Q_BYTES, 16, 1024);
-            const uint64_t dk0 = sdesc_sw128(sKV, 16, 1024);
+            const uint64_t dq0 = L::SW64 ? sdesc_sw64(sQ) : sdesc_sw128(sQ, 16, 1024);
+            const uint64_t dq1 = L::SW64 ? sdesc_sw64(sQ + L::Q_BYTES)
+                                         : sdesc_sw128(sQ + L::Q_BYTES, 16, 1024);
+            const uint64_t dk0 = L::SW64 ? sdesc_sw64(sKV) : sdesc_sw128(sKV, 16, 1024);
             const uint64_t dv0 = F8 ? sdesc_sw128(sKV, 16, 1024)     // V^T: K-major
                                     : sdesc_sw128(sKV, L::HALF_BYTES, 1024);
             const uint32_t stage_step = uint32_t(L::KV_BYTES >> 4);
@@ -1023,8 +1027,9 @@ fa_status launch(const void* q, const void* k, const void* v, void* o, float* ls
 // ---------------------------------------------------------------------------
 // FP8 forward: V^T pre-pass, E4M3 tensor maps, kernel launch.
 // ---------------------------------------------------------------------------
-constexpr int FP8_D = 128;
-constexpr int FP8_NS = 8;                        // 16 KiB K or V^T tiles: 8 ring stages
+// Ring stages: 16 KiB K or V^T tiles at d = 128 (8 stages), 8 KiB at d = 64 (16).
+constexpr int FP8_NS_128 = 8;
+constexpr int FP8_NS_64 = 16;
 
 long long fp8_npad(int N) { return ((long long)N + fa::BN - 1) / fa::BN * fa::BN; }
 
@@ -1061,23 +1066,24 @@ __global__ void __launch_bounds__(256) transpose_v_e4m3(const uint8_t* __restric
 }
 
 // 4-D E4M3 tensor map (inner, rows, H, B), contiguous, byte strides; box
-// (128, box_rows, 1, 1) in 128-byte swizzle.
+// (box_inner, box_rows, 1, 1) in 128-byte swizzle, or 64-byte swizzle for a
+// 64-byte inner box.
 fa_status encode_map_e4m3(CUtensorMap* map, const void* base, long long inner, long long rows,
-                          int H, int B, int box_rows) {
+                          int H, int B, int box_inner, int box_rows) {
     const cuuint64_t dims[4] = {cuuint64_t(inner), cuuint64_t(rows), cuuint64_t(H), cuuint64_t(B)};
     const cuuint64_t strides[3] = {cuuint64_t(inner), cuuint64_t(inner * rows),
                                    cuuint64_t(inner * rows * H)};
-    const cuuint32_t box[4] = {128u, cuuint32_t(box_rows), 1u, 1u};
+    const cuuint32_t box[4] = {cuuint32_t(box_inner), cuuint32_t(box_rows), 1u, 1u};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          box_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_UNSUPPORTED;
 }
 
-size_t fp8_workspace_bytes(long long BH, int N) {
-    return size_t(FA_DYNAMIC_WORKSPACE_BYTES) + size_t(BH * FP8_D * fp8_npad(N));
+size_t fp8_workspace_bytes(long long BH, int N, int d) {
+    return size_t(FA_DYNAMIC_WORKSPACE_BYTES) + size_t(BH * d * fp8_npad(N));
 }
 
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -1216,9 +1222,9 @@ fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, vo
 }
 
 size_t fa_fwd_fp8_workspace_bytes(int B, int H, int N, int d) {
-    if (B < 1 || H < 1 || N < 1 || d != FP8_D) return 0;
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
     if ((long long)B * H > 0x7fffffffLL || N > (1 << 30)) return 0;
-    return fp8_workspace_bytes((long long)B * H, N);
+    return fp8_workspace_bytes((long long)B * H, N, d);
 }
 
 fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B,
@@ -1230,12 +1236,12 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, fl
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
     for (float x : {scale, descale_q, descale_k, descale_v})
         if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
-    if (d != FP8_D) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     const long long BH = (long long)B * H;
     if (BH > 0xffffLL || N > (1 << 30)) return FA_ERR_UNSUPPORTED;   // grid.y of the V^T pass
     if (((long long)N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS * BH > (1LL << 30))
         return FA_ERR_UNSUPPORTED;
-    if (workspace_bytes < fp8_workspace_bytes(BH, N)) return FA_ERR_INVALID_ARG;
+    if (workspace_bytes < fp8_workspace_bytes(BH, N, d)) return FA_ERR_INVALID_ARG;
     if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(o, 16) ||
         !aligned(lse, 4) || !aligned(workspace, 256))
         return FA_ERR_MISALIGNED;
@@ -1247,15 +1253,23 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, fl
     uint8_t* vt = static_cast<uint8_t*>(workspace) + FA_DYNAMIC_WORKSPACE_BYTES;
     const long long npad = fp8_npad(N);
     CUtensorMap mq, mk, mv;
-    if (encode_map_e4m3(&mq, q8, FP8_D, N, H, B, fa::BM) != FA_OK ||
-        encode_map_e4m3(&mk, k8, FP8_D, N, H, B, fa::BN) != FA_OK ||
-        encode_map_e4m3(&mv, vt, npad, FP8_D, H, B, FP8_D) != FA_OK)
+    if (encode_map_e4m3(&mq, q8, d, N, H, B, d, fa::BM) != FA_OK ||
+        encode_map_e4m3(&mk, k8, d, N, H, B, d, fa::BN) != FA_OK ||
+        encode_map_e4m3(&mv, vt, npad, d, H, B, 128, d) != FA_OK)
         return FA_ERR_UNSUPPORTED;
-    transpose_v_e4m3<FP8_D><<<dim3(unsigned(npad / 64), unsigned(BH)), 256, 0, s>>>(
-        static_cast<const uint8_t*>(v8), vt, N, npad);
+    if (d == 64)
+        transpose_v_e4m3<64><<<dim3(unsigned(npad / 64), unsigned(BH)), 256, 0, s>>>(
+            static_cast<const uint8_t*>(v8), vt, N, npad);
+    else
+        transpose_v_e4m3<128><<<dim3(unsigned(npad / 64), unsigned(BH)), 256, 0, s>>>(
+            static_cast<const uint8_t*>(v8), vt, N, npad);
     const float scale_log2 = scale * descale_q * descale_k * 1.4426950408889634f;
-    const Strides3 ost{(long long)H * N * FP8_D, (long long)N * FP8_D, (long long)FP8_D};
-    return launch_kernel<FP8_D, FP8_NS, true>(mq, mk, mv, o, lse, B, H, N, ost, causal, scale_log2,
+    const Strides3 ost{(long long)H * N * d, (long long)N * d, (long long)d};
+    if (d == 64)
+        return launch_kernel<64, FP8_NS_64, true>(mq, mk, mv, o, lse, B, H, N, ost, causal,
+                                                  scale_log2, descale_v, sched, s, dev,
+                                                  4000ull * 1000000ull, 0);
+    return launch_kernel<128, FP8_NS_128, true>(mq, mk, mv, o, lse, B, H, N, ost, causal, scale_log2,
                                               descale_v, sched, s, dev, 4000ull * 1000000ull, 0);
 }
 

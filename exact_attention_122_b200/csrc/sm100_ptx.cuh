@@ -280,6 +280,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
+// Shared-memory matrix descriptor, 64-byte swizzle (CU_TENSOR_MAP_SWIZZLE_64B
+// layout: 8 rows of 64 bytes per 512-byte atom), K-major: stride byte offset
+// = 512 between 8-row groups, layout type 4.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t(1) << 16;                          // leading byte offset (unused when swizzled)
+    d |= uint64_t((512u >> 4) & 0x3FFFu) << 32;
+    d |= uint64_t(1) << 46;
+    d |= uint64_t(4) << 61;
+    return d;
+}
+
 // Instruction descriptor for kind::f8f6f4 with E4M3 A and B (format code 0),
 // fp32 accumulator, both operands K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {

@@ -219,7 +219,7 @@ size_t fa_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
  * cores (page "FlashAttention: The GPU Memory Hack That Changed Everything",
  * "FlashAttention-3: Hopper Architecture": attention run in FP8 precision).
  *
- *  q8, k8, v8 : E4M3 codes [B][H][N][d], contiguous, d = 128; the values are
+ *  q8, k8, v8 : E4M3 codes [B][H][N][d], contiguous, d in {64, 128}; the values are
  *               code * descale_q (resp. _k, _v), one scale per tensor.
  *  o          : bf16 [B][H][N][d];  lse : fp32 [B][H][N], natural-log units
  *               of scale * (descale_q q8) . (descale_k k8).
@@ -233,7 +233,7 @@ size_t fa_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
  * the workspace so both tensor-core operands are K-major.
  * Errors: FA_ERR_INVALID_ARG (NULL pointers, sizes < 1, bad causal flag, scale
  * or descale not finite and > 0, workspace too small), FA_ERR_UNSUPPORTED
- * (d != 128, B*H > 65535, sizes beyond the limits of fa_fwd, device not
+ * (d not 64 or 128, B*H > 65535, sizes beyond the limits of fa_fwd, device not
  * sm_100), FA_ERR_MISALIGNED (inputs or o not 16-byte aligned, lse not
  * 4-byte aligned, workspace not 256-byte aligned), FA_ERR_NO_DEVICE,
  * FA_ERR_LAUNCH.

@@ -194,8 +194,8 @@ def test_fp8_argument_validation_and_workspace_size():
         for bad in (0.0, -1.0, float("nan"), float("inf")):
             a = list(ok); a[i] = bad
             assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_INVALID_ARG
-    a = list(ok); a[8] = 64
-    assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_UNSUPPORTED                    # d = 64
+    a = list(ok); a[8] = 96
+    assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_UNSUPPORTED                    # d = 96
     a = list(ok); a[5] = 300; a[6] = 300
     assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_UNSUPPORTED                    # B*H > 65535
     a = list(ok); a[15] = fa.fp8_workspace_bytes(2, 3, 1000, 128) - 1
@@ -206,7 +206,8 @@ def test_fp8_argument_validation_and_workspace_size():
     assert fa.fa_fwd_fp8_raw(*a) == fa.FA_ERR_MISALIGNED
     # workspace: 256-byte work counter + V^T (B*H*d*Npad bytes, Npad = N rounded up to 128)
     assert fa.fp8_workspace_bytes(2, 3, 1000, 128) == 256 + 6 * 128 * 1024
-    assert fa.fp8_workspace_bytes(2, 3, 1000, 64) == 0
+    assert fa.fp8_workspace_bytes(2, 3, 1000, 64) == 256 + 6 * 64 * 1024
+    assert fa.fp8_workspace_bytes(2, 3, 1000, 96) == 0
 
 
 def test_bwd_debug_validates_inject():

@@ -83,6 +83,18 @@ def test_fp8_ragged(fa, N, causal):
     compare(fa, 1, 2, N, causal, seed=500 + N)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 100, 256, 257, 1000, 2048])
+def test_fp8_ragged_d64(fa, N, causal):
+    compare(fa, 1, 2, N, causal, seed=600 + N, d=64)
+
+
+def test_fp8_d64_workload_shapes(fa):
+    # the BERT- and GPT-2-shaped workloads in FP8
+    compare(fa, 8, 12, 512, False, seed=1222, d=64)
+    compare(fa, 8, 12, 1024, True, seed=1223, d=64)
+
+
 def test_fp8_batch_heads(fa):
     compare(fa, 2, 3, 1000, True, seed=61)
 
@@ -148,7 +160,7 @@ def test_fp8_argument_errors_on_device(fa):
     assert fa.fa_fwd_fp8_raw(*args, ws.numel() - 1, s) == fa.FA_ERR_INVALID_ARG
     bad = list(args); bad[1] = p + 8
     assert fa.fa_fwd_fp8_raw(*bad, ws.numel(), s) == fa.FA_ERR_MISALIGNED
-    bad = list(args); bad[8] = 64
+    bad = list(args); bad[8] = 96
     assert fa.fa_fwd_fp8_raw(*bad, ws.numel(), s) == fa.FA_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert fa.device_status()[0] == fa.FA_OK
