@@ -20,7 +20,7 @@ EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_dynami
                     "fa_fwd_fp8",
                     "fa_fwd_debug",
                     "fa_get_device_status", "fa_status_string", "fa_last_cuda_error", "fa_version")
-DECODE_MAX_QUERIES = 16                # FA_DECODE_MAX_QUERIES
+DECODE_MAX_QUERIES = 1 << 30           # FA_DECODE_MAX_QUERIES
 DECODE_MAX_SPLITS = 256                # FA_DECODE_MAX_SPLITS
 DYNAMIC_WORKSPACE_BYTES = 256          # FA_DYNAMIC_WORKSPACE_BYTES in include/fa.h
 

@@ -5,7 +5,7 @@
 // N_q FLOPs per byte of K and V, far below the B200 ridge, so the path is
 // bound by streaming K and V from HBM once.  From N_q = 5 on, the FP32 pipes
 // could not keep up with that stream (16 queries need about 100 TFLOP/s at
-// the copy bandwidth), so decode_mma_kernel pads the queries to 16 rows and
+// the copy bandwidth), so decode_mma_kernel takes the queries in blocks of 16 rows and
 // forms both products with the warp-level m16n8k16 bf16 tensor-core MMA.  The
 // same kernel serves N_q <= 4: its coalesced, double-buffered cp.async
 // staging streams K and V faster than the earlier lane-per-key CUDA-core
@@ -44,8 +44,8 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ---------------------------------------------------------------------------
-// Split kernel, 1 <= N_q <= 16: the queries are padded to
-// MQ = 16 rows (m16n8k16).  Each warp streams 16-key tiles of its split
+// Split kernel: a CTA takes one key split of one (batch, head) and one block
+// of MQ = 16 query rows (m16n8k16; the last block padded with zero rows).  Each warp streams 16-key tiles of its split
 // through two shared-memory stages (cp.async), forms S = Q K^T with K
 // fragments from ldmatrix, runs the online softmax on the accumulator
 // fragments (rows lane/4 and lane/4 + 8, a quad per row), repacks P as the A
@@ -120,7 +120,10 @@ __global__ void __launch_bounds__(THREADS)
     using S = MmaSmem<D>;
     extern __shared__ __align__(16) unsigned char dsm[];
     const uint32_t sb = smem_u32(dsm);
-    const int split = blockIdx.x, bh = blockIdx.y;
+    // Query blocks vary fastest in the launch order, so the CTAs that read
+    // the same keys run together and all but one take K and V from L2.
+    const int split = blockIdx.y, bh = blockIdx.z;
+    const int q0 = blockIdx.x * MQ;                   // first query row of this CTA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int k0 = split * chunk;
     const int k1 = min(Nk, k0 + chunk);
@@ -133,7 +136,7 @@ __global__ void __launch_bounds__(THREADS)
     for (int e = threadIdx.x; e < MQ * D / 8; e += THREADS) {
         const int row = e / (D / 8), c = e - (e / (D / 8)) * (D / 8);
         uint4 x = make_uint4(0u, 0u, 0u, 0u);
-        if (row < Nq) x = *reinterpret_cast<const uint4*>(Qb + size_t(row) * D + c * 8);
+        if (q0 + row < Nq) x = *reinterpret_cast<const uint4*>(Qb + size_t(q0 + row) * D + c * 8);
         *reinterpret_cast<uint4*>(dsm + S::OFF_Q + row * S::ROW + c * 16) = x;
     }
     __syncthreads();
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int key = kt + nb * 8 + cq + (c & 1);
-                const int row = r0 + (c >> 1) * 8;
+                const int row = q0 + r0 + (c >> 1) * 8;
                 const bool ok = key < k1 && (!causal || key <= row + off);
                 sc[nb][c] = ok ? sc[nb][c] * scale_log2 : -INFINITY;
             }
@@ -265,19 +268,20 @@ __global__ void __launch_bounds__(THREADS)
             sm_o[(warp * MQ + r0 + (c >> 1) * 8) * D + nb * 8 + cq + (c & 1)] = o[nb][c];
     __syncthreads();
     for (int e = threadIdx.x; e < MQ * D; e += THREADS) {
-        const int i = e / D, t = e - (e / D) * D;
+        const int il = e / D, t = e - (e / D) * D;    // local row, column
+        const int i = q0 + il;
         if (i >= Nq) continue;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < WARPS; ++w) M = fmaxf(M, sm_m[w * MQ + i]);
+        for (int w = 0; w < WARPS; ++w) M = fmaxf(M, sm_m[w * MQ + il]);
         float L = 0.f, acc = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < WARPS; ++w) {
-                const float mw = sm_m[w * MQ + i];
+                const float mw = sm_m[w * MQ + il];
                 const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
-                L += sm_l[w * MQ + i] * f;
-                acc += sm_o[(w * MQ + i) * D + t] * f;
+                L += sm_l[w * MQ + il] * f;
+                acc += sm_o[(w * MQ + il) * D + t] * f;
             }
         }
         const size_t row = (size_t(split) * BH + bh) * Nq + i;
@@ -311,20 +315,26 @@ __global__ void __launch_bounds__(D)
     if (t == 0) LSE[r] = W > 0.f ? M + logf(W) : -INFINITY;
 }
 
-int auto_splits(long long BH, int Nk) {
-    // At least 8 splits (measured on B200 with B*H = 512, Nk = 32K: 1 split
-    // reaches 47 % of the copy bandwidth, 8 or more splits 83 %), enough to
-    // cover the SMs twice for small B*H, at least 512 keys per split, at
-    // most 64 splits.
-    long long s = (2 * 148 + BH - 1) / BH;
-    if (s < 8) s = 8;
+int auto_splits(long long BH, int Nq, int Nk) {
+    // Enough CTAs (splits x B*H x query blocks) to cover the SMs twice; with
+    // a single query block at least 8 splits (measured on B200 with
+    // B*H = 512, Nk = 32K: 1 split reaches 47 % of the copy bandwidth, 8 or
+    // more splits 83 %); at least 512 keys per split, at most 64 splits.
+    const long long qblocks = (Nq + MQ - 1) / MQ;
+    long long s = (2 * 148 + BH * qblocks - 1) / (BH * qblocks);
+    if (qblocks == 1 && s < 8) s = 8;
     const long long by_keys = (Nk + 511) / 512;
     if (s > by_keys) s = by_keys;
     if (s > 64) s = 64;
     return int(s < 1 ? 1 : s);
 }
 
+// Above this many queries the persistent tiled kernel (128-row tcgen05 tiles)
+// does the work; it needs only its 256-byte work counter as workspace.
+constexpr int TILED_MIN_NQ = 33;
+
 size_t workspace_bytes(long long BH, int Nq, int d, int splits) {
+    if (Nq >= TILED_MIN_NQ) return FA_DYNAMIC_WORKSPACE_BYTES;
     const size_t rows = size_t(BH) * Nq;
     const size_t o_bytes = size_t(splits) * rows * d * sizeof(float);
     const size_t l_bytes = size_t(splits) * rows * sizeof(float);
@@ -363,7 +373,7 @@ size_t fa_fwd_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d, int nu
         num_splits > FA_DECODE_MAX_SPLITS)
         return 0;
     const long long BH = (long long)B * H;
-    const int splits = num_splits ? num_splits : fa_decode::auto_splits(BH, Nk);
+    const int splits = num_splits ? num_splits : fa_decode::auto_splits(BH, Nq, Nk);
     return fa_decode::workspace_bytes(BH, Nq, d, splits);
 }
 
@@ -383,8 +393,13 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
     if (!al(q, 16) || !al(k, 16) || !al(v, 16) || !al(o, 16) || !al(lse, 4) || !al(workspace, 256))
         return FA_ERR_MISALIGNED;
     const long long BH = (long long)B * H;
-    const int splits = num_splits ? num_splits : fa_decode::auto_splits(BH, Nk);
+    const int splits = num_splits ? num_splits : fa_decode::auto_splits(BH, Nq, Nk);
     if (ws_bytes < fa_decode::workspace_bytes(BH, Nq, d, splits)) return FA_ERR_INVALID_ARG;
+    if (Nq >= fa_decode::TILED_MIN_NQ)
+        return static_cast<fa_status>(fa_internal::forward_qk(q, k, v, o, lse, B, H, Nq, Nk, d,
+                                                               causal, scale,
+                                                               static_cast<int*>(workspace),
+                                                               stream));
 
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -407,7 +422,7 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
                                             ((o_bytes + 255) & ~size_t(255)));
     const float sl2 = scale * 1.4426950408889634f;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const dim3 grid{unsigned(used), unsigned(BH), 1u};
+    const dim3 grid{unsigned((Nq + fa_decode::MQ - 1) / fa_decode::MQ), unsigned(used), unsigned(BH)};
     e = d == 64 ? fa_decode::launch_mma<64>(grid, s, q, k, v, opart, lpart, int(BH), Nq, Nk,
                                             causal, sl2, chunk)
                 : fa_decode::launch_mma<128>(grid, s, q, k, v, opart, lpart, int(BH), Nq, Nk,

@@ -211,9 +211,13 @@ __device__ __forceinline__ int unit_index(int k, int cta, int ctas) {
     return k * ctas + ((k & 1) ? (ctas - 1 - cta) : cta);
 }
 
-__device__ __forceinline__ Unit decode_unit(int i, int BH, int N, int causal, int hg) {
-    const int nq2 = (N + UNIT_ROWS - 1) / UNIT_ROWS;
-    const int nkb = (N + BN - 1) / BN;
+// N_q query rows and N_k keys per (batch, head); with causal masking query i
+// may see key j iff j <= i + N_k - N_q (the queries are the last N_q
+// positions), so a sub-tile's last row r sees keys up to r + N_k - N_q.
+__device__ __forceinline__ Unit decode_unit(int i, int BH, int Nq, int Nk, int causal, int hg) {
+    const int nq2 = (Nq + UNIT_ROWS - 1) / UNIT_ROWS;
+    const int nkb = (Nk + BN - 1) / BN;
+    const int off = Nk - Nq;
     const int per_group = hg * nq2;
     const int g = i / per_group;
     const int r = i - g * per_group;
@@ -224,8 +228,8 @@ __device__ __forceinline__ Unit decode_unit(int i, int BH, int N, int causal, in
     const int qb2 = causal ? (nq2 - 1 - level) : level;
     w.r0 = qb2 * UNIT_ROWS;
     if (causal) {
-        w.nb0 = min(w.r0 / BN + 1, nkb);
-        w.nb1 = min(w.r0 / BN + 2, nkb);
+        w.nb0 = min((w.r0 + BM - 1 + off) / BN + 1, nkb);
+        w.nb1 = min((w.r0 + 2 * BM - 1 + off) / BN + 1, nkb);
     } else {
         w.nb0 = nkb;
         w.nb1 = nkb;
@@ -329,7 +333,8 @@ template <int D, int NS, bool F8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ Og,
-                  float* __restrict__ LSEg, int BH, int H, int N, int causal, float scale_log2,
+                  float* __restrict__ LSEg, int BH, int H, int Nq, int Nk, int causal,
+                  float scale_log2,
                   int hg, long long o_sb, long long o_sh, long long o_sn, int* __restrict__ sched,
                   unsigned long long watchdog_ns, int inject, float o_scale) {
     using L = Layout<D, NS, F8>;
@@ -350,9 +355,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int nq2 = (N + UNIT_ROWS - 1) / UNIT_ROWS;
+    const int nq2 = (Nq + UNIT_ROWS - 1) / UNIT_ROWS;
     const int num_units = nq2 * BH;
-    const int nkb = (N + BN - 1) / BN;
+    const int nkb = (Nk + BN - 1) / BN;
+    const int koff = Nk - Nq;                  // causal: key j allowed for row i iff j <= i + koff
     const Watchdog wd_in{abort_flag, watchdog_ns};
     // Unit queue.  Static schedule (sched == nullptr): every role walks the
     // same boustrophedon sequence.  Dynamic schedule: the producer claims
@@ -443,7 +449,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (u >= num_units) u = -1;
                 }
                 if (u < 0) break;
-                const Unit w = decode_unit(u, BH, N, causal, hg);
+                const Unit w = decode_unit(u, BH, Nq, Nk, causal, hg);
                 const int wb = w.bh / H, wh = w.bh - (w.bh / H) * H;   // batch, head
                 if (!wait_phase(bar(L::B_Q_EMPTY), (units & 1u) ^ 1u, wd, ROLE_PRODUCER, u)) {
                     ok = false;
@@ -528,7 +534,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int kq = 0; ok; ++kq, ++units) {
                 const int u = next_unit_consumer(kq, ok, ROLE_MMA);
                 if (u < 0) break;
-                const Unit w = decode_unit(u, BH, N, causal, hg);
+                const Unit w = decode_unit(u, BH, Nq, Nk, causal, hg);
                 if (!wait_phase(bar(L::B_Q_FULL), units & 1u, wd, ROLE_MMA, u)) { ok = false; break; }
                 uint32_t sK = cons % NS;
                 if (!wait_phase(bar(L::B_KV_FULL + sK), (cons / NS) & 1u, wd, ROLE_MMA, u)) {
@@ -633,7 +639,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kq = 0; ok; ++kq) {
             const int u = next_unit_consumer(kq, ok, ROLE_SOFTMAX);
             if (u < 0) break;
-            const Unit w = decode_unit(u, BH, N, causal, hg);
+            const Unit w = decode_unit(u, BH, Nq, Nk, causal, hg);
             const int a = w.r0 + t * BM;             // first row of this sub-tile
             const int row = a + wr;
             const int nb = t == 0 ? w.nb0 : w.nb1;
@@ -651,13 +657,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
                 }
-                // Mask: keys beyond N on the last tile; keys above the
-                // diagonal on a sub-tile's diagonal tile.
-                const bool tail = (j == nkb - 1) && (N % BN != 0);
-                const bool diag = causal && (j == a / BN);
+                // Mask: keys beyond N_k on the last tile; causal: keys past
+                // the row's limit on the tiles that cross the sub-tile's
+                // first limit (the diagonal).
+                const bool tail = (j == nkb - 1) && (Nk % BN != 0);
+                const bool diag = causal && (j * BN + BN - 1 > a + koff);
                 if (tail || diag) {
-                    const int lim_tail = N - j * BN;           // key c allowed iff c < lim_tail
-                    const int lim_diag = row - j * BN;         // key c allowed iff c <= lim_diag
+                    const int lim_tail = Nk - j * BN;          // key c allowed iff c < lim_tail
+                    const int lim_diag = row + koff - j * BN;  // key c allowed iff c <= lim_diag
 #pragma unroll
                     for (int c = 0; c < BN; ++c) {
                         const bool bad = (c >= lim_tail) || (causal && c > lim_diag);
@@ -723,7 +730,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             float inv_l = 1.f / l;
             if constexpr (F8) inv_l *= o_scale;
-            const bool store = row < N;
+            const bool store = row < Nq;
             const int wb = w.bh / H, wh = w.bh - (w.bh / H) * H;     // batch, head
             __nv_bfloat16* orow = Og + wb * o_sb + wh * o_sh + (long long)(store ? row : 0) * o_sn;
             uint32_t ro[D];
@@ -750,7 +757,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     dst[v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
-            if (store) LSEg[size_t(w.bh) * N + row] = (m + log2f(l)) * 0.69314718055994530942f;
+            if (store) LSEg[size_t(w.bh) * Nq + row] = (m + log2f(l)) * 0.69314718055994530942f;
             tc_fence_before();
             mbar_arrive(bar(L::B_O_EMPTY + t));
         }
@@ -881,9 +888,10 @@ namespace {
 // groups).  Decisions are cached per shape.
 struct HgKey {
     long long BH;
-    int N, D, causal, grid;
+    int Nq, Nk, D, causal, grid;
     bool operator==(const HgKey& o) const {
-        return BH == o.BH && N == o.N && D == o.D && causal == o.causal && grid == o.grid;
+        return BH == o.BH && Nq == o.Nq && Nk == o.Nk && D == o.D && causal == o.causal &&
+               grid == o.grid;
     }
 };
 std::mutex g_hg_mutex;
@@ -891,9 +899,10 @@ HgKey g_hg_keys[64];
 long long g_hg_vals[64];
 int g_hg_count = 0;
 
-double snake_imbalance(long long BH, int N, int causal, long long hg, int grid) {
-    const long long nq2 = (N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
-    const long long nkb = (N + fa::BN - 1) / fa::BN;
+double snake_imbalance(long long BH, int Nq, int Nk, int causal, long long hg, int grid) {
+    const long long nq2 = (Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+    const long long nkb = (Nk + fa::BN - 1) / fa::BN;
+    const long long off = Nk - Nq;
     const long long units = nq2 * BH;
     std::vector<long long> load(size_t(grid), 0);
     const long long per_group = hg * nq2;
@@ -903,8 +912,9 @@ double snake_imbalance(long long BH, int N, int causal, long long hg, int grid) 
         const long long gh = std::min(hg, BH - g * hg);
         const long long level = r / gh;
         const long long r0 = (causal ? (nq2 - 1 - level) : level) * fa::UNIT_ROWS;
-        const long long nb0 = causal ? std::min(r0 / fa::BN + 1, nkb) : nkb;
-        const long long nb1 = causal ? std::min(r0 / fa::BN + 2, nkb) : nkb;
+        const long long nb0 = causal ? std::min((r0 + fa::BM - 1 + off) / fa::BN + 1, nkb) : nkb;
+        const long long nb1 =
+            causal ? std::min((r0 + 2 * fa::BM - 1 + off) / fa::BN + 1, nkb) : nkb;
         const long long k = i / grid, c = i - k * grid;
         load[size_t((k & 1) ? (grid - 1 - c) : c)] += nb0 + nb1 + 2;   // +2: per-unit overhead
     }
@@ -916,19 +926,19 @@ double snake_imbalance(long long BH, int N, int causal, long long hg, int grid) 
     return double(mx) * grid / double(sum);
 }
 
-long long choose_head_group(long long BH, int N, int D, int causal, int grid) {
-    const HgKey key{BH, N, D, causal, grid};
+long long choose_head_group(long long BH, int Nq, int Nk, int D, int causal, int grid) {
+    const HgKey key{BH, Nq, Nk, D, causal, grid};
     {
         std::lock_guard<std::mutex> lk(g_hg_mutex);
         for (int i = 0; i < g_hg_count; ++i)
             if (g_hg_keys[i] == key) return g_hg_vals[i];
     }
-    const long long kv_head_bytes = 2LL * N * D * 2;
+    const long long kv_head_bytes = 2LL * Nk * D * 2;
     long long best = BH;
     double best_cost = 1e30;
     // Bound the replay work for very large problems: beyond ~4M units the
     // assignment statistics no longer depend on hg, so all heads form one group.
-    const long long units = ((N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS) * BH;
+    const long long units = ((Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS) * BH;
     if (units <= (4LL << 20)) {
         for (long long hg = 1;; hg = std::min(hg * 2, BH)) {
             const double ws = double(hg * kv_head_bytes);
@@ -936,7 +946,7 @@ long long choose_head_group(long long BH, int N, int D, int causal, int grid) {
                              : ws <= 32.0 * (1 << 20) ? 0.03
                              : ws <= 64.0 * (1 << 20) ? 0.06
                              : ws <= 128.0 * (1 << 20) ? 0.09 : 0.12;
-            const double cost = snake_imbalance(BH, N, causal, hg, grid) * (1.0 + pen);
+            const double cost = snake_imbalance(BH, Nq, Nk, causal, hg, grid) * (1.0 + pen);
             if (cost < best_cost - 1e-9) {
                 best_cost = cost;
                 best = hg;
@@ -955,9 +965,9 @@ long long choose_head_group(long long BH, int N, int D, int causal, int grid) {
 // attribute setup, head-group choice, dynamic-schedule counter reset.
 template <int D, int NS, bool F8>
 fa_status launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                        void* o, float* lse, int B, int H, int N, const Strides3& ost, int causal,
-                        float scale_log2, float o_scale, int* sched, cudaStream_t stream, int dev,
-                        unsigned long long watchdog_ns, int inject) {
+                        void* o, float* lse, int B, int H, int Nq, int Nk, const Strides3& ost,
+                        int causal, float scale_log2, float o_scale, int* sched,
+                        cudaStream_t stream, int dev, unsigned long long watchdog_ns, int inject) {
     using L = fa::Layout<D, NS, F8>;
     using I = Instance<D, NS, F8>;
     auto kern = fa::fa_fwd_kernel<D, NS, F8>;
@@ -977,16 +987,16 @@ fa_status launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     // so such a build is refused rather than launched.
     if (I::regs[dev] != fa::REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
     const long long BH = (long long)B * H;
-    const long long nq2 = (N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+    const long long nq2 = (Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
     const long long units = nq2 * BH;
     const int grid = int(units < g_dev[dev].sm_count ? units : g_dev[dev].sm_count);
     // Static schedule: group size from the replayed assignment.  Dynamic
     // schedule: CTAs claim units greedily, so balance no longer depends on the
     // group size; groups then hold about 16 MiB of K/V (all heads when the
     // whole K/V fits in 32 MiB).
-    const long long kv_head_bytes = 2LL * N * D * L::EB;
+    const long long kv_head_bytes = 2LL * Nk * D * L::EB;
     long long hg = sched ? ((BH * kv_head_bytes <= (32LL << 20)) ? BH : (16LL << 20) / kv_head_bytes)
-                         : choose_head_group(BH, N, D, causal, grid);
+                         : choose_head_group(BH, Nq, Nk, D, causal, grid);
 #ifdef FA_HEAD_GROUP
     hg = FA_HEAD_GROUP;
 #endif
@@ -999,7 +1009,7 @@ fa_status launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
         }
     }
     kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o),
-                                                     lse, int(BH), H, N, causal, scale_log2,
+                                                     lse, int(BH), H, Nq, Nk, causal, scale_log2,
                                                      int(hg), ost.b, ost.h, ost.n, sched,
                                                      watchdog_ns, inject, o_scale);
     cudaError_t e = cudaGetLastError();
@@ -1012,16 +1022,16 @@ fa_status launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
 
 template <int D, int NS>
 fa_status launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                 int N, const Strides3 (&st)[4], int causal, float scale, int* sched,
+                 int Nq, int Nk, const Strides3 (&st)[4], int causal, float scale, int* sched,
                  cudaStream_t stream, int dev, unsigned long long watchdog_ns, int inject) {
     CUtensorMap mq, mk, mv;
-    if (encode_map(&mq, q, D, N, H, B, st[0]) != FA_OK ||
-        encode_map(&mk, k, D, N, H, B, st[1]) != FA_OK ||
-        encode_map(&mv, v, D, N, H, B, st[2]) != FA_OK)
+    if (encode_map(&mq, q, D, Nq, H, B, st[0]) != FA_OK ||
+        encode_map(&mk, k, D, Nk, H, B, st[1]) != FA_OK ||
+        encode_map(&mv, v, D, Nk, H, B, st[2]) != FA_OK)
         return FA_ERR_UNSUPPORTED;
     const float scale_log2 = scale * 1.4426950408889634f;
-    return launch_kernel<D, NS, false>(mq, mk, mv, o, lse, B, H, N, st[3], causal, scale_log2, 1.f,
-                                       sched, stream, dev, watchdog_ns, inject);
+    return launch_kernel<D, NS, false>(mq, mk, mv, o, lse, B, H, Nq, Nk, st[3], causal, scale_log2,
+                                       1.f, sched, stream, dev, watchdog_ns, inject);
 }
 
 // ---------------------------------------------------------------------------
@@ -1087,35 +1097,39 @@ size_t fp8_workspace_bytes(long long BH, int N, int d) {
 }
 
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                   int N, int d, const long long* strides12, int causal, float scale, int* sched,
-                   void* stream, unsigned watchdog_ms, int inject) {
+                   int Nq, int Nk, int d, const long long* strides12, int causal, float scale,
+                   int* sched, void* stream, unsigned watchdog_ms, int inject) {
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (causal && Nq > Nk) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
     if (inject != 0 && inject != 1) return FA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-    if ((long long)B * H > 0x7fffffffLL || N > (1 << 30)) return FA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0x7fffffffLL || Nq > (1 << 30) || Nk > (1 << 30))
+        return FA_ERR_UNSUPPORTED;
     // The kernel numbers 256-row units with 32-bit ints (and the dynamic
     // schedule claims up to units + grid indices).
-    if (((long long)N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS * B * H > (1LL << 30))
+    if (((long long)Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS * B * H > (1LL << 30))
         return FA_ERR_UNSUPPORTED;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
         return FA_ERR_MISALIGNED;
     // Strides: q, k, v, o in that order, each (batch, head, sequence) in
-    // elements; NULL means contiguous [B][H][N][d].
+    // elements; NULL means contiguous [B][H][N][d] (N = N_q for q and o, N_k
+    // for k and v).
     Strides3 st[4];
     for (int i = 0; i < 4; ++i) {
+        const int n = (i == 1 || i == 2) ? Nk : Nq;
         if (strides12) {
             st[i] = Strides3{strides12[3 * i], strides12[3 * i + 1], strides12[3 * i + 2]};
         } else {
-            st[i] = Strides3{(long long)H * N * d, (long long)N * d, (long long)d};
+            st[i] = Strides3{(long long)H * n * d, (long long)n * d, (long long)d};
         }
         // The stride of a dimension of size 1 is never used; frameworks may
         // report any value there, so it is replaced by a valid one.
         if (B == 1) st[i].b = d;
         if (H == 1) st[i].h = d;
-        if (N == 1) st[i].n = d;
+        if (n == 1) st[i].n = d;
         const long long v3[3] = {st[i].b, st[i].h, st[i].n};
         for (long long x : v3) {
             if (x < d) return FA_ERR_INVALID_ARG;               // rows may not overlap within a head dim
@@ -1131,13 +1145,20 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     const unsigned long long wd_ns = (watchdog_ms ? watchdog_ms : 4000u) * 1000000ull;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (d == 64)
-        return launch<64, 8>(q, k, v, o, lse, B, H, N, st, causal, scale, sched, s, dev, wd_ns,
+        return launch<64, 8>(q, k, v, o, lse, B, H, Nq, Nk, st, causal, scale, sched, s, dev, wd_ns,
                              inject);
-    return launch<128, 4>(q, k, v, o, lse, B, H, N, st, causal, scale, sched, s, dev, wd_ns,
+    return launch<128, 4>(q, k, v, o, lse, B, H, Nq, Nk, st, causal, scale, sched, s, dev, wd_ns,
                           inject);
 }
 
 }  // namespace
+
+int fa_internal::forward_qk(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                            int* counter, void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, nullptr, causal, scale, counter, stream, 0,
+                    0);
+}
 
 // ===========================================================================
 // Allocation-free variant of fa_fwd_dynamic (fa_fwd_dynamic_noalloc).
@@ -1173,14 +1194,14 @@ extern "C" {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int N, int d, int causal, float scale, void* stream) {
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, nullptr, causal, scale, nullptr, stream, 0, 0);
+    return fwd_impl(q, k, v, o, lse, B, H, N, N, d, nullptr, causal, scale, nullptr, stream, 0, 0);
 }
 
 fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int H, int N, int d, const long long* strides, int causal, float scale,
                          void* stream) {
     if (!strides) return FA_ERR_INVALID_ARG;
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale, nullptr, stream, 0, 0);
+    return fwd_impl(q, k, v, o, lse, B, H, N, N, d, strides, causal, scale, nullptr, stream, 0, 0);
 }
 
 fa_status fa_fwd_dynamic(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -1189,7 +1210,7 @@ fa_status fa_fwd_dynamic(const void* q, const void* k, const void* v, void* o, f
     if (!workspace) return FA_ERR_INVALID_ARG;
     if (workspace_bytes < FA_DYNAMIC_WORKSPACE_BYTES) return FA_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return FA_ERR_MISALIGNED;
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale,
+    return fwd_impl(q, k, v, o, lse, B, H, N, N, d, strides, causal, scale,
                     static_cast<int*>(workspace), stream, 0, 0);
 }
 
@@ -1217,7 +1238,7 @@ fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, vo
     }
     // Same launch path as fa_fwd_dynamic: the counter is cleared on `stream`
     // before the kernel runs.
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, strides, causal, scale,
+    return fwd_impl(q, k, v, o, lse, B, H, N, N, d, strides, causal, scale,
                     static_cast<int*>(ns.ptr), stream, 0, 0);
 }
 
@@ -1266,17 +1287,18 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, fl
     const float scale_log2 = scale * descale_q * descale_k * 1.4426950408889634f;
     const Strides3 ost{(long long)H * N * d, (long long)N * d, (long long)d};
     if (d == 64)
-        return launch_kernel<64, FP8_NS_64, true>(mq, mk, mv, o, lse, B, H, N, ost, causal,
+        return launch_kernel<64, FP8_NS_64, true>(mq, mk, mv, o, lse, B, H, N, N, ost, causal,
                                                   scale_log2, descale_v, sched, s, dev,
                                                   4000ull * 1000000ull, 0);
-    return launch_kernel<128, FP8_NS_128, true>(mq, mk, mv, o, lse, B, H, N, ost, causal, scale_log2,
+    return launch_kernel<128, FP8_NS_128, true>(mq, mk, mv, o, lse, B, H, N, N, ost, causal,
+                                                scale_log2,
                                               descale_v, sched, s, dev, 4000ull * 1000000ull, 0);
 }
 
 fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int H, int N, int d, int causal, float scale, void* stream,
                        unsigned watchdog_ms, int inject) {
-    return fwd_impl(q, k, v, o, lse, B, H, N, d, nullptr, causal, scale, nullptr, stream,
+    return fwd_impl(q, k, v, o, lse, B, H, N, N, d, nullptr, causal, scale, nullptr, stream,
                     watchdog_ms, inject);
 }
 

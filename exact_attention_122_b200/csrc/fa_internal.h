@@ -21,6 +21,12 @@ int current_device(int* dev, int* sm_count);
 int encode_bhnd_map(CUtensorMap* map, const void* base, int d, int N, int H, int B, long long sb,
                     long long sh, long long sn, int box_rows);
 
+// The persistent tiled forward for N_q query rows against N_k keys (causal:
+// the queries are the last N_q positions), dynamic schedule with its 4-byte
+// work counter at `counter` (device memory).  Returns an fa_status.
+int forward_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int Nq, int Nk, int d, int causal, float scale, int* counter, void* stream);
+
 // Reads and clears the backward kernels' watchdog word (after the caller has
 // synchronised): 0 when no wait ran out.  Returns a cudaError_t.
 int take_bwd_status(unsigned* word);

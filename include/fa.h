@@ -162,8 +162,8 @@ fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, vo
                                  int B, int H, int N, int d, const long long* strides, int causal,
                                  float scale, void* stream);
 
-/* Largest number of query rows per (batch, head) fa_fwd_decode accepts. */
-#define FA_DECODE_MAX_QUERIES 16
+/* Largest number of query rows per (batch, head) fa_fwd_decode accepts (2^30). */
+#define FA_DECODE_MAX_QUERIES 1073741824
 /* Largest explicit split count of fa_fwd_decode. */
 #define FA_DECODE_MAX_SPLITS 256
 
@@ -175,28 +175,32 @@ fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, vo
 size_t fa_fwd_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits);
 
 /*
- * fa_fwd_decode -- exact attention for few queries against a long key
- * sequence (decoding), split over the keys.
+ * fa_fwd_decode -- exact attention for N_q queries against N_k keys with
+ * N_q != N_k: decoding (few queries) and prefill against a cache.
  *
  * Same operation as fa_fwd with separate lengths: q, o bf16 [B][H][Nq][d]
  * and k, v bf16 [B][H][Nk][d], contiguous; lse float [B][H][Nq].  With
  * causal = 1 the queries are the last Nq positions of the key sequence:
- * query i may see key j iff j <= i + Nk - Nq (needs Nq <= Nk).  The keys
- * are cut into `num_splits` ranges (0 = automatic) processed in parallel;
- * each range keeps the online-softmax running state of the page "Flash
- * attention optimization" ("The fix: tile the computation ..."), and a
- * second kernel merges the ranges with that page's rescale-and-merge rule.
- * This shape is bound by reading K and V once from device memory.  The
- * queries are padded to 16 rows for warp-level bf16 tensor-core MMAs, and P
- * is rounded to bf16 before the P V product, as in fa_fwd.
+ * query i may see key j iff j <= i + Nk - Nq (needs Nq <= Nk).
+ *  - Nq <= 32: the keys are cut into `num_splits` ranges (0 = automatic)
+ *    processed in parallel, each keeping the online-softmax running state of
+ *    the page "Flash attention optimization" ("The fix: tile the computation
+ *    ..."); a second kernel merges the ranges with that page's
+ *    rescale-and-merge rule.  The queries go in blocks of 16 rows (one CTA
+ *    each, the last block padded) to warp-level bf16 tensor-core MMAs.  This
+ *    shape is bound by reading K and V once from device memory.
+ *  - Nq > 32: the persistent tiled kernel of fa_fwd_dynamic (128-row tcgen05
+ *    tiles), with the causal alignment above; num_splits is ignored and the
+ *    workspace holds only its work counter.
+ * In both, P is rounded to bf16 before the P V product, as in fa_fwd.
  *
  *  Nq          : 1 .. FA_DECODE_MAX_QUERIES.
  *  Nk          : >= 1 (>= Nq when causal), <= 2^30;  B*H <= 65535.
  *  num_splits  : 0 (automatic) .. FA_DECODE_MAX_SPLITS.
  *  workspace   : device memory owned by the caller, 256-byte aligned, at
  *                least fa_fwd_decode_workspace_bytes(...) bytes; it holds
- *                the per-split partial results and must not be shared by
- *                calls that may run at the same time.
+ *                the per-split partial results (or the work counter) and
+ *                must not be shared by calls that may run at the same time.
  * Errors: FA_ERR_INVALID_ARG (NULL pointers or workspace, sizes < 1,
  * causal with Nq > Nk, bad scale or split count, workspace too small),
  * FA_ERR_UNSUPPORTED (d not 64/128, Nq > FA_DECODE_MAX_QUERIES, sizes beyond

@@ -135,8 +135,8 @@ def test_decode_argument_validation_and_workspace_size():
     ok = (P, P, P, P, P, 2, 3, 1, 1000, 128, 0, 0.1, 0, W, 1 << 30, 0)
     a = list(ok); a[13] = 0
     assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_INVALID_ARG                 # NULL workspace
-    a = list(ok); a[7] = 17
-    assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_UNSUPPORTED                 # Nq > 16
+    a = list(ok); a[7] = (1 << 30) + 1
+    assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_UNSUPPORTED                 # Nq > 2^30
     a = list(ok); a[7] = 8; a[8] = 4; a[10] = 1
     assert fa.fa_fwd_decode_raw(*a) == fa.FA_ERR_INVALID_ARG                 # causal with Nq > Nk
     a = list(ok); a[12] = 257
@@ -151,6 +151,9 @@ def test_decode_argument_validation_and_workspace_size():
     assert fa.decode_workspace_bytes(2, 3, 4, 1000, 128, 5) == 5 * 6 * 4 * 128 * 4 + 5 * 6 * 4 * 4
     assert fa.decode_workspace_bytes(2, 3, 4, 1000, 128, 300) == 0
     assert fa.decode_workspace_bytes(2, 3, 4, 1000, 128, 0) > 0
+    # Nq > 32 runs the tiled kernel: only its 256-byte work counter
+    assert fa.decode_workspace_bytes(2, 3, 33, 1000, 128, 0) == 256
+    assert fa.decode_workspace_bytes(2, 3, 32, 1000, 128, 1) == 32 * 6 * 128 * 4 + 32 * 6 * 4
     assert fa.fa_fwd_decode_raw(*ok) == fa.FA_ERR_NO_DEVICE                  # valid: stops at the device query
 
 

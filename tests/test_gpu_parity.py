@@ -359,9 +359,15 @@ DECODE_CASES = [
     (2, 4, 1, 4096, 128, False, 0), (2, 4, 1, 4097, 64, True, 0), (1, 8, 16, 3000, 128, True, 0),
     (3, 2, 7, 130, 64, True, 3), (1, 2, 5, 5, 128, True, 0), (1, 1, 1, 1, 64, False, 0),
     (2, 3, 3, 1000, 128, True, 1), (2, 3, 3, 1000, 128, False, 9), (1, 4, 12, 20000, 128, True, 0),
-    # tensor-core kernel (5 <= Nq <= 16): ragged key tiles, few keys, explicit splits
+    # ragged key tiles, few keys, explicit splits
     (2, 3, 9, 777, 64, False, 0), (1, 2, 16, 33, 64, True, 2), (1, 3, 6, 4096, 128, False, 5),
     (1, 2, 16, 1, 128, False, 0), (2, 2, 8, 8, 128, True, 0), (1, 2, 13, 2049, 128, True, 0),
+    # several 16-row query blocks
+    (1, 2, 17, 500, 128, True, 0), (1, 2, 32, 3000, 64, True, 0), (2, 1, 29, 999, 64, False, 2),
+    # N_q > 32: the tiled kernel with N_q != N_k (prefill against a cache)
+    (2, 2, 40, 3000, 64, True, 0), (1, 3, 100, 100, 128, True, 3), (1, 2, 300, 4096, 128, True, 0),
+    (2, 1, 65, 999, 64, False, 2), (1, 1, 1024, 1024, 64, True, 0), (1, 2, 257, 1000, 128, True, 0),
+    (2, 2, 700, 2000, 128, False, 0), (1, 2, 1000, 5000, 64, True, 0),
 ]
 
 
@@ -375,10 +381,11 @@ def test_decode_parity(fa, B, H, Nq, Nk, d, causal, splits):
     check(o, lse, O_ref, L_ref, f"decode B={B} H={H} Nq={Nq} Nk={Nk} d={d} causal={causal}")
 
 
-def test_decode_matches_square_last_rows(fa):
+@pytest.mark.parametrize("Nq", [8, 300])
+def test_decode_matches_square_last_rows(fa, Nq):
     """Decode of the last Nq queries equals the last Nq rows of the square
     causal problem computed by fa_fwd (within the parity tolerance)."""
-    B, H, N, d, Nq = 1, 4, 2000, 128, 8
+    B, H, N, d = 1, 4, 2000, 128
     q, k, v = synth.draw_qkv(B, H, N, d, seed=61)
     qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
     o_sq, l_sq = fa.fa_fwd(qd, kd, vd, causal=True)

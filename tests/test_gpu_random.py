@@ -94,7 +94,7 @@ def test_random_fp8(fa, case):
 def test_random_decode(fa, case):
     i, B, H, N, d, causal, scale = case
     rng = np.random.default_rng(9000 + i)
-    Nq = int(rng.integers(1, 17))
+    Nq = int(rng.choice([int(rng.integers(1, 17)), int(rng.integers(17, 200))]))
     Nk = max(N, Nq) if causal else N
     q, k, v = synth.draw_decode_qkv(B, H, Nq, Nk, d, seed=9000 + i)
     splits = int(rng.choice([0, 1, 3, 7]))
