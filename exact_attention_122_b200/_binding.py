@@ -17,7 +17,7 @@ FA_ERR_NO_DEVICE = 6
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_strided", "fa_fwd_dynamic", "fa_fwd_dynamic_noalloc",
                     "fa_fwd_decode_workspace_bytes", "fa_fwd_decode", "fa_bwd_workspace_bytes",
                     "fa_bwd", "fa_bwd_strided", "fa_bwd_debug", "fa_fwd_fp8_workspace_bytes",
-                    "fa_fwd_fp8",
+                    "fa_fwd_fp8", "fa_fwd_host_workspace_bytes", "fa_fwd_host",
                     "fa_fwd_debug",
                     "fa_get_device_status", "fa_status_string", "fa_last_cuda_error", "fa_version")
 DECODE_MAX_QUERIES = 1 << 30           # FA_DECODE_MAX_QUERIES
@@ -74,6 +74,10 @@ def library() -> ctypes.CDLL:
     lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, vp, ctypes.c_size_t,
                                vp]
     lib.fa_fwd_fp8.restype = i
+    lib.fa_fwd_host_workspace_bytes.argtypes = [i, i, i, i]
+    lib.fa_fwd_host_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, ctypes.c_size_t, vp]
+    lib.fa_fwd_host.restype = i
     lib.fa_fwd_debug.argtypes = fwd_args + [u, i]
     lib.fa_fwd_debug.restype = i
     lib.fa_get_device_status.argtypes = [vp, ctypes.POINTER(u)]
@@ -320,6 +324,65 @@ def fa_fwd_fp8(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float,
                             s.cuda_stream)
     if st != FA_OK:
         raise FaError(st, "fa_fwd_fp8")
+    return out, lse
+
+
+def host_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(library().fa_fwd_host_workspace_bytes(B, H, N, d))
+
+
+def fa_fwd_host_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int,
+                    N: int, d: int, causal: int, scale: float, ws_ptr: int, ws_bytes: int,
+                    stream_ptr: int) -> int:
+    """Direct call of fa_fwd_host (host q/k/v/o/lse); returns the fa_status code."""
+    return library().fa_fwd_host(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal, scale,
+                                 ws_ptr, ws_bytes, stream_ptr)
+
+
+def fa_fwd_host(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+                workspace=None, stream=None, device=None):
+    """O, LSE of exact attention for bf16 (B, H, N, d) tensors in HOST memory
+    (page-locked for overlap: ``tensor.pin_memory()``), through fa_fwd_host:
+    chunks of heads are copied to ``device``, computed and copied back with
+    the transfers overlapped.  ``out`` / ``lse`` (host, allocated pinned when
+    not given) hold the results once ``stream`` (default: the current torch
+    stream of ``device``) has been synchronised.  ``workspace`` is a device
+    tensor of at least host_workspace_bytes(B, H, N, d) bytes, allocated when
+    not given."""
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not (t.device.type == "cpu" and t.dtype == torch.bfloat16 and t.dim() == 4
+                and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 host tensor (B, H, N, d)")
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one shape (B, H, N, d)")
+    B, H, N, d = q.shape
+    device = torch.device(device) if device is not None else torch.device(
+        "cuda", torch.cuda.current_device())
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
+    if not (out.device.type == "cpu" and out.dtype == torch.bfloat16 and out.shape == q.shape
+            and out.is_contiguous()):
+        raise ValueError("out must be a contiguous bf16 host tensor shaped like q")
+    if not (lse.device.type == "cpu" and lse.dtype == torch.float32
+            and tuple(lse.shape) == (B, H, N) and lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 host tensor of shape (B, H, N)")
+    need = host_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    with torch.cuda.device(device):
+        s = stream if stream is not None else torch.cuda.current_stream(device)
+        st = fa_fwd_host_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), B, H, N, d, 1 if causal else 0, float(scale),
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             s.cuda_stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_host")
     return out, lse
 
 

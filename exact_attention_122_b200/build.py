@@ -13,7 +13,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SOURCES = [os.path.join(PKG, "csrc", "fa_fwd_sm100.cu"),
            os.path.join(PKG, "csrc", "fa_decode_sm100.cu"),
-           os.path.join(PKG, "csrc", "fa_bwd_sm100.cu")]
+           os.path.join(PKG, "csrc", "fa_bwd_sm100.cu"),
+           os.path.join(PKG, "csrc", "fa_host.cu")]
 HEADERS = [os.path.join(ROOT, "include", "fa.h"), os.path.join(PKG, "csrc", "fa_internal.h"),
            os.path.join(PKG, "csrc", "sm100_ptx.cuh")]
 LIB = os.path.join(PKG, "libfa_b200.so")

@@ -162,6 +162,47 @@ fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, vo
                                  int B, int H, int N, int d, const long long* strides, int causal,
                                  float scale, void* stream);
 
+/*
+ * fa_fwd_host_workspace_bytes -- device workspace fa_fwd_host needs: two
+ * slots, each holding Q, K, V, O and LSE of one chunk of heads plus a work
+ * counter.  Returns 0 for sizes fa_fwd_host would reject.
+ */
+size_t fa_fwd_host_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * fa_fwd_host -- fa_fwd on tensors that live in HOST memory, with the
+ * transfers overlapped with the attention.  A deployment variant (the pages
+ * have no counterpart): the operation and the result are those of fa_fwd.
+ *
+ * The B*H heads are cut into up to 16 chunks of whole heads.  Chunk c is
+ * copied into slot c % 2 of `workspace`, computed there by the persistent
+ * forward kernel (dynamic schedule), and its O and LSE are copied back, on
+ * three streams internal to the library, so the copy in of one chunk, the
+ * attention of the previous one and the copy out of the one before run at
+ * the same time.  With page-locked host memory the call is bound by the
+ * host <-> device link; pageable memory gives the same result, serialised.
+ *
+ *  q, k, v  : HOST pointers, bf16 [B][H][N][d], contiguous (any alignment).
+ *  o        : HOST pointer, bf16 [B][H][N][d];  lse : HOST pointer, float
+ *             [B][H][N], natural log.  All five are owned by the caller and
+ *             must stay valid, and o/lse unread, until `stream` is
+ *             synchronised.
+ *  workspace: DEVICE memory owned by the caller, 256-byte aligned, at least
+ *             fa_fwd_host_workspace_bytes(...) bytes; calls that share it
+ *             must be ordered (the same stream, or events).
+ *  stream   : the call starts after the work queued on it and the stream
+ *             waits for the last copy back, so synchronising it (or an event
+ *             recorded on it after the call) covers the whole call.
+ * Other arguments as fa_fwd.  Errors: as fa_fwd (no alignment rule on the
+ * host buffers), plus FA_ERR_INVALID_ARG for a NULL or too small workspace
+ * and FA_ERR_MISALIGNED for a workspace that is not 256-byte aligned.  Every
+ * check runs before anything is enqueued; FA_ERR_LAUNCH if a copy or a
+ * launch is refused.
+ */
+fa_status fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int N, int d, int causal, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
 /* Largest number of query rows per (batch, head) fa_fwd_decode accepts (2^30). */
 #define FA_DECODE_MAX_QUERIES 1073741824
 /* Largest explicit split count of fa_fwd_decode. */

@@ -234,3 +234,43 @@ def test_bwd_strided_argument_validation():
     assert fa.fa_bwd_strided_raw(*base, bad, *tail) == fa.FA_ERR_MISALIGNED
     bad = list(st); bad[12] = 1 << 40                                    # dout batch stride too large
     assert fa.fa_bwd_strided_raw(*base, bad, *tail) == fa.FA_ERR_UNSUPPORTED
+
+
+def _host_ws(B, H, N, d):
+    """fa_fwd_host's workspace: two slots of one chunk (ceil(B*H/16) heads) each,
+    Q, K, V, O (bf16) and LSE (fp32) padded to 256 bytes, plus a 256-byte counter."""
+    up = lambda x: (x + 255) // 256 * 256
+    hc = -(-(B * H) // 16)
+    return 2 * (4 * up(hc * N * d * 2) + up(hc * N * 4) + 256)
+
+
+def test_host_argument_validation_and_workspace_size():
+    W = 1 << 22
+    need = fa.host_workspace_bytes(2, 3, 1000, 128)
+    assert need == _host_ws(2, 3, 1000, 128) == 2056704
+    assert fa.host_workspace_bytes(2, 32, 8192, 128) == _host_ws(2, 32, 8192, 128)
+    assert fa.host_workspace_bytes(1, 1, 33, 64) == _host_ws(1, 1, 33, 64)
+    assert fa.host_workspace_bytes(2, 3, 1000, 96) == 0
+    assert fa.host_workspace_bytes(0, 3, 1000, 64) == 0
+    ok = [P + 1, P + 3, P + 5, P + 7, P + 2, 2, 3, 1000, 128, 1, 0.1, W, need, 0]
+    assert fa.fa_fwd_host_raw(*ok) == fa.FA_ERR_NO_DEVICE   # host buffers need no alignment
+    for i in (0, 1, 2, 3, 4, 11):                            # NULL pointer or workspace
+        a = list(ok); a[i] = 0
+        assert fa.fa_fwd_host_raw(*a) == fa.FA_ERR_INVALID_ARG
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        a = list(ok); a[10] = bad
+        assert fa.fa_fwd_host_raw(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok); a[9] = 2
+    assert fa.fa_fwd_host_raw(*a) == fa.FA_ERR_INVALID_ARG  # causal flag
+    a = list(ok); a[7] = 0
+    assert fa.fa_fwd_host_raw(*a) == fa.FA_ERR_INVALID_ARG  # N < 1
+    a = list(ok); a[8] = 96
+    assert fa.fa_fwd_host_raw(*a) == fa.FA_ERR_UNSUPPORTED  # d = 96
+    a = list(ok); a[5] = 1 << 16; a[6] = 1 << 16
+    assert fa.fa_fwd_host_raw(*a) == fa.FA_ERR_UNSUPPORTED  # B*H = 2^32
+    a = list(ok); a[5] = 1 << 15; a[6] = 1 << 15
+    assert fa.fa_fwd_host_raw(*a) == fa.FA_ERR_UNSUPPORTED  # 2^30 heads * 4 units > 2^30
+    a = list(ok); a[12] = need - 1
+    assert fa.fa_fwd_host_raw(*a) == fa.FA_ERR_INVALID_ARG  # workspace too small
+    a = list(ok); a[11] = W + 16
+    assert fa.fa_fwd_host_raw(*a) == fa.FA_ERR_MISALIGNED   # workspace not 256-byte aligned
