@@ -80,6 +80,25 @@ fa_status launch_error(cudaError_t e) {
     return FA_ERR_LAUNCH;
 }
 
+// Makes `s` wait for everything queued so far on the three internal streams
+// (each wait takes the event's latest record, so one event serves all three).
+cudaError_t join(HostPipe& p, cudaStream_t s) {
+    cudaError_t e = cudaSuccess;
+    for (cudaStream_t x : {p.s_in, p.s_cmp, p.s_out}) {
+        if (e == cudaSuccess) e = cudaEventRecord(p.end, x);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, p.end, 0);
+    }
+    return e;
+}
+
+// A failure after the first enqueue: the caller's stream still waits for the
+// copies already queued, so freeing the buffers after synchronising it is safe.
+fa_status fail_after_enqueue(HostPipe& p, cudaStream_t s, int status, cudaError_t e) {
+    if (e != cudaSuccess) fa_internal::set_last_cuda_error(int(e));   // else already recorded
+    join(p, s);
+    return static_cast<fa_status>(status);
+}
+
 }  // namespace
 
 extern "C" {
@@ -148,13 +167,13 @@ fa_status fa_fwd_host(const void* q, const void* k, const void* v, void* o, floa
         // attention: after the inputs, and after chunk ci-2's outputs left the slot
         if (e == cudaSuccess) e = cudaStreamWaitEvent(p.s_cmp, p.in_done[slot], 0);
         if (e == cudaSuccess && ci >= kSlots) e = cudaStreamWaitEvent(p.s_cmp, p.out_done[slot], 0);
-        if (e != cudaSuccess) return launch_error(e);
+        if (e != cudaSuccess) return fail_after_enqueue(p, s, FA_ERR_LAUNCH, e);
         const int st = fa_internal::forward_qk(base, base + c.off_k, base + c.off_v,
                                                base + c.off_o,
                                                reinterpret_cast<float*>(base + c.off_l), 1,
                                                int(hn), N, N, d, causal, scale,
                                                reinterpret_cast<int*>(base + c.off_ctr), p.s_cmp);
-        if (st != FA_OK) return static_cast<fa_status>(st);
+        if (st != FA_OK) return fail_after_enqueue(p, s, st, cudaSuccess);
         e = cudaEventRecord(p.cmp_done[slot], p.s_cmp);
         // copy out
         if (e == cudaSuccess) e = cudaStreamWaitEvent(p.s_out, p.cmp_done[slot], 0);
@@ -165,13 +184,13 @@ fa_status fa_fwd_host(const void* q, const void* k, const void* v, void* o, floa
             e = cudaMemcpyAsync(reinterpret_cast<unsigned char*>(lse) + size_t(h0) * N * 4,
                                 base + c.off_l, lbytes, cudaMemcpyDefault, p.s_out);
         if (e == cudaSuccess) e = cudaEventRecord(p.out_done[slot], p.s_out);
-        if (e != cudaSuccess) return launch_error(e);
+        if (e != cudaSuccess) return fail_after_enqueue(p, s, FA_ERR_LAUNCH, e);
     }
     // The caller's stream waits for the last copy out, which follows every
     // other operation of the call.
     e = cudaEventRecord(p.end, p.s_out);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, p.end, 0);
-    if (e != cudaSuccess) return launch_error(e);
+    if (e != cudaSuccess) return fail_after_enqueue(p, s, FA_ERR_LAUNCH, e);
     return FA_OK;
 }
 

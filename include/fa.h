@@ -17,11 +17,14 @@
  * order; O is rounded to bf16 once at the end.
  *
  * Conventions shared by every entry point:
- *  - Pointers named q, k, v, o, lse are DEVICE pointers owned by the caller.
- *    The library never allocates, frees or retains them.
+ *  - Pointers named q, k, v, o, lse are DEVICE pointers owned by the caller
+ *    (fa_fwd_host alone takes HOST pointers there).  The library never
+ *    allocates, frees or retains them.
  *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
- *    the legacy default stream) and the call returns without synchronising.
- *    Results are valid once the caller has synchronised that stream.
+ *    the legacy default stream) and the call returns without synchronising
+ *    (fa_fwd_host on pageable host memory excepted: CUDA copies pageable
+ *    memory synchronously).  Results are valid once the caller has
+ *    synchronised that stream.
  *  - Arguments are validated before anything is enqueued; an invalid call
  *    returns an error status and has no side effect.
  *  - Calls are thread-safe.  One call per stream at a time may run on a
@@ -187,17 +190,19 @@ size_t fa_fwd_host_workspace_bytes(int B, int H, int N, int d);
  *             [B][H][N], natural log.  All five are owned by the caller and
  *             must stay valid, and o/lse unread, until `stream` is
  *             synchronised.
- *  workspace: DEVICE memory owned by the caller, 256-byte aligned, at least
- *             fa_fwd_host_workspace_bytes(...) bytes; calls that share it
- *             must be ordered (the same stream, or events).
+ *  workspace: DEVICE memory of the current device, owned by the caller,
+ *             256-byte aligned, at least fa_fwd_host_workspace_bytes(...)
+ *             bytes; calls that share it must be ordered (the same stream,
+ *             or events).
  *  stream   : the call starts after the work queued on it and the stream
  *             waits for the last copy back, so synchronising it (or an event
  *             recorded on it after the call) covers the whole call.
  * Other arguments as fa_fwd.  Errors: as fa_fwd (no alignment rule on the
  * host buffers), plus FA_ERR_INVALID_ARG for a NULL or too small workspace
  * and FA_ERR_MISALIGNED for a workspace that is not 256-byte aligned.  Every
- * check runs before anything is enqueued; FA_ERR_LAUNCH if a copy or a
- * launch is refused.
+ * check runs before anything is enqueued.  FA_ERR_LAUNCH if a copy or a
+ * launch is refused part-way; `stream` then still waits for the chunks
+ * already queued, and o / lse hold only part of the result.
  */
 fa_status fa_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int H, int N, int d, int causal, float scale, void* workspace,
