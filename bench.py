@@ -3,9 +3,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one exact-attention forward (one fa_fwd_dynamic launch, or fa_fwd
-with --schedule static) over one batch of
-the long-context causal workload (B=2, H=32, N=8192, d=128, bf16, seeded
+A step is one exact-attention forward (one fa_fwd_dynamic launch: the
+"auto" schedule picks it for this size; --schedule static times fa_fwd) over
+one batch of the long-context causal workload (B=2, H=32, N=8192, d=128, bf16, seeded
 N(0,1) inputs), inputs resident in HBM.  FLOPs per step: 4*B*H*N^2*d / 2.
 Prints one JSON line (rank 0).
 
@@ -23,6 +23,12 @@ reading K and V once: its metric is effective HBM GB/s.
 ``--sweep`` instead prints one line per sequence length of the page's
 "Try It Yourself" sweep (B=1, H=32, d=128, causal, N = 512..8192), device
 timed like the main line; it is an extra curve, not the headline number.
+
+A workload whose step moves less than twice the 126 MB L2 (``--workload``
+1-3, the sweep below N = 8192) is timed differently: the launches cycle
+through enough copies of the buffers that none finds its inputs in L2, L2
+is flushed before the timed region, and the launches are replayed from one
+CUDA graph, since eager launches of a few microseconds would time the host.
 """
 
 from __future__ import annotations
@@ -300,7 +306,8 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, args.gpus, args.schedule),
+        "config": workload_config(w, args.gpus, bench_schedule(args.schedule, w),
+                                  rotation_copies(w.algorithmic_bytes, args.steps)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -309,12 +316,87 @@ def run_reference(args, w):
     return 0
 
 
-def workload_config(w: synth.Workload, n_gpus: int, schedule: str = "dynamic"):
+L2_BYTES = 126 * 1000 * 1000    # B200 L2 capacity
+
+
+def rotation_copies(step_bytes: int, steps: int) -> int:
+    """Copies of one step's buffers that the timed launches cycle through so
+    that no launch finds its inputs in L2: 1 when a step alone moves at least
+    twice the L2 capacity; otherwise enough copies that at least twice the L2
+    capacity streams between two uses of one copy, but never more copies than
+    launches (each copy is then used once, after an L2 flush)."""
+    if step_bytes >= 2 * L2_BYTES:
+        return 1
+    return max(2, min(steps, math.ceil(2 * L2_BYTES / step_bytes) + 1))
+
+
+def l2_note(step_bytes: int, copies: int) -> str:
+    if copies == 1:
+        return f"one step moves {step_bytes / 1e6:.0f} MB > 2 x 126 MB L2; no flush"
+    return (f"one step moves {step_bytes / 1e6:.1f} MB < 2 x 126 MB L2: launches cycle through "
+            f"{copies} copies of the buffers and L2 is flushed (252 MB write) before the timed "
+            f"region; launches replayed from one CUDA graph")
+
+
+B200_SM_COUNT = 148
+
+
+def bench_schedule(schedule: str, w: synth.Workload, sm_count: int | None = None) -> str:
+    """The forward schedule a line uses ("auto" resolved the way fa_fwd
+    resolves it; the reference arm, which needs no GPU, assumes a B200)."""
+    from exact_attention_122_b200._binding import resolve_schedule
+
+    return resolve_schedule(schedule, w.B, w.H, w.N, sm_count or B200_SM_COUNT)
+
+
+def require_beyond_l2(step_bytes: int, steps: int, mode: str) -> None:
+    """The --bwd and --fp8 lines time eager launches without an L2 flush, which
+    is valid only when one step moves at least twice the L2 capacity."""
+    if rotation_copies(step_bytes, steps) != 1:
+        raise SystemExit(f"{mode} times workloads whose step moves >= {2 * L2_BYTES / 1e6:.0f} MB "
+                         f"(this one moves {step_bytes / 1e6:.1f} MB): use --workload 4 or 5")
+
+
+def fwd_kernel_name(d: int, fp8: bool = False) -> str:
+    ns = {(128, False): 4, (64, False): 8, (128, True): 8, (64, True): 16}[(d, fp8)]
+    return f"fa_fwd_kernel<{d},{ns}{',true' if fp8 else ''}>"
+
+
+def time_graph(launch, n_launch: int, replays: int, stream, local: int, sync_all):
+    """Capture launch(0..n_launch-1) into one CUDA graph, replay it once
+    untimed, flush L2, then time `replays` replays with CUDA events on
+    `stream`.  Returns (total ms, clock summary)."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n_launch):
+            launch(i)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=stream.device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        flush.zero_()
+    sync_all()
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(replays):
+                g.replay()
+            e1.record(stream)
+        sync_all()
+    total = e0.elapsed_time(e1)
+    del g
+    return total, clocks.summary()
+
+
+def workload_config(w: synth.Workload, n_gpus: int, schedule: str = "dynamic", copies: int = 1):
     return {"workload": w.name, "schedule": schedule,
             "B_per_gpu": w.B, "H": w.H, "N": w.N, "d": w.d,
             "causal": w.causal, "scale": w.scale, "global_batch": w.B * n_gpus, "seq_len": w.N,
             "parallelism": f"independent batches x{n_gpus}" if n_gpus > 1 else "single GPU",
-            "l2": f"inputs {3 * w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB > 126 MB L2; no flush"}
+            "l2": l2_note(w.algorithmic_bytes, copies)}
 
 
 # ---------------------------------------------------------------------------
@@ -336,6 +418,7 @@ def run_ours(args, w):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
+    sched = bench_schedule(args.schedule, w, torch.cuda.get_device_properties(dev).multi_processor_count)
     q, k, v = synth.draw_qkv(w.B, w.H, w.N, w.d, rank_seed(w.seed, rank), w.qk_std)
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
     od = torch.empty_like(qd)
@@ -344,7 +427,7 @@ def run_ours(args, w):
 
     def step():
         fa.fa_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=od, lse=lsed, stream=stream,
-                  schedule=args.schedule)
+                  schedule=sched)
 
     def sync_all():
         torch.cuda.synchronize(dev)
@@ -358,25 +441,44 @@ def run_ours(args, w):
     if st != fa.FA_OK:
         raise SystemExit(f"kernel status {fa.status_string(st)} {word:#x}")
 
-    # --- device-timed region: K launches, per-launch events on the launch stream
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    t_begin = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    sync_all()
-    with ClockSampler(local) as clocks:
-        with torch.cuda.stream(stream):
-            t_begin.record(stream)
-            for i in range(args.steps):
-                starts[i].record(stream)
-                step()
-                ends[i].record(stream)
-            t_end.record(stream)
+    copies = rotation_copies(w.algorithmic_bytes, args.steps)
+    if copies == 1:
+        # --- device-timed region: K launches, per-launch events on the launch stream
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        t_begin = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
         sync_all()
-    total_ms = t_begin.elapsed_time(t_end)
-    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(total_ms, dev)
-    avg_launch_ms = max_over_ranks(sum(launch_ms) / len(launch_ms), dev)
+        with ClockSampler(local) as clocks:
+            with torch.cuda.stream(stream):
+                t_begin.record(stream)
+                for i in range(args.steps):
+                    starts[i].record(stream)
+                    step()
+                    ends[i].record(stream)
+                t_end.record(stream)
+            sync_all()
+        clock_summary = clocks.summary()
+        total_ms = t_begin.elapsed_time(t_end)
+        launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        total_ms = max_over_ranks(total_ms, dev)
+        avg_launch_ms = max_over_ranks(sum(launch_ms) / len(launch_ms), dev)
+    else:
+        # --- a workload smaller than L2: the K launches cycle through copies of
+        # the buffers and run from one CUDA graph (eager launches of a few
+        # microseconds would time the host); per launch = total / K.
+        bufs = [(qd, kd, vd, od, lsed)] + [
+            (qd.clone(), kd.clone(), vd.clone(), torch.empty_like(od), torch.empty_like(lsed))
+            for _ in range(copies - 1)]
+
+        def launch(i):
+            a = bufs[i % copies]
+            fa.fa_fwd(a[0], a[1], a[2], causal=w.causal, scale=w.scale, out=a[3], lse=a[4],
+                      stream=stream, schedule=sched)
+
+        total_ms, clock_summary = time_graph(launch, args.steps, 1, stream, local, sync_all)
+        total_ms = max_over_ranks(total_ms, dev)
+        avg_launch_ms = total_ms / args.steps
     st, word = fa.device_status(stream.cuda_stream)
     if st != fa.FA_OK:
         raise SystemExit(f"kernel status {fa.status_string(st)} {word:#x}")
@@ -424,18 +526,18 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w, world, args.schedule),
+        "config": workload_config(w, world, sched, copies),
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "frac_of_sustained": (achieved / peak_sustained) if peak_sustained else None,
-                     "kernel": "fa_fwd_kernel<128,4>", "avg_launch_ms": avg_launch_ms},
+                     "kernel": fwd_kernel_name(w.d), "avg_launch_ms": avg_launch_ms},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "entry": "fa_fwd_host",
                 "ms_per_step": e2e_ms / e2e_steps},
         "gpu_launches": args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clock_summary,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, secs, desc = time_oracle_sample(w, q, k, v, target_s=args.cpu_seconds)
@@ -514,6 +616,9 @@ def run_bwd(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     w = synth.workload(args.workload)
+    elems = w.B * w.H * w.N * w.d
+    step_bytes = 8 * 2 * elems + 4 * w.B * w.H * w.N    # Q,K,V,O,dO in, dQ,dK,dV out; LSE
+    require_beyond_l2(step_bytes, args.steps, "--bwd")
     q, k, v = (t.to(dev) for t in synth.workload_qkv(w))
     dout = synth.draw_dout(w.B, w.H, w.N, w.d, seed=w.seed).to(dev)
     stream = torch.cuda.Stream(device=dev)
@@ -553,7 +658,7 @@ def run_bwd(args):
             "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                        "causal": w.causal, "flops_per_step": flops,
-                       "l2": "inputs 537 MB > 126 MB L2; no flush"},
+                       "l2": l2_note(step_bytes, 1)},
             "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s",
                          "frac": value / peak,
                          "traffic": load_traffic(w.name + "_bwd", BWD_KERNEL_SOURCE),
@@ -574,6 +679,8 @@ def run_fp8(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     w = synth.workload(args.workload)
+    step_bytes = 5 * w.B * w.H * w.N * w.d + 4 * w.B * w.H * w.N   # E4M3 Q,K,V in, bf16 O out; LSE
+    require_beyond_l2(step_bytes, args.steps, "--fp8")
     (q8, k8, v8), (sq, sk, sv) = synth.draw_qkv_fp8(w.B, w.H, w.N, w.d, seed=w.seed,
                                                      qk_std=w.qk_std)
     q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
@@ -611,7 +718,7 @@ def run_fp8(args):
             "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "dtype": "e4m3", "data": "synthetic",
             "config": {"workload": w.name + "_fp8", "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                       "causal": w.causal, "l2": "inputs 268 MB > 126 MB L2; no flush"},
+                       "causal": w.causal, "l2": l2_note(step_bytes, 1)},
             "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s",
                          "frac": value / peak, "traffic": load_traffic(w.name + "_fp8"),
                          "traffic_kernel": "fa_fwd_kernel<128, 8, true>",
@@ -631,27 +738,54 @@ def run_sweep(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.Stream(device=dev)
     peak, _, peak_src = load_peaks()
+
+    def sync_all():
+        torch.cuda.synchronize(dev)
+
     for N in synth.SWEEP_SEQ_LENS:
         w = synth.sweep_workload(N)
+        sched = bench_schedule(args.schedule, w, torch.cuda.get_device_properties(dev).multi_processor_count)
         q, k, v = (t.to(dev) for t in synth.workload_qkv(w))
         o = torch.empty_like(q)
         lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
         # at least ~200 ms of timed work per length, and at least args.steps launches
         steps = max(args.steps, int(0.2 / max(w.flops / 1.0e15, 1e-6)))
+        copies = rotation_copies(w.algorithmic_bytes, steps)
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
                 fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream,
-                          schedule=args.schedule)
+                          schedule=sched)
+        sync_all()
+        if copies == 1:
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize(dev)
-            e0.record(stream)
-            for _ in range(steps):
-                fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream,
-                          schedule=args.schedule)
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1) / steps
+            with ClockSampler(0) as clocks:
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    for _ in range(steps):
+                        fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, stream=stream,
+                                  schedule=sched)
+                    e1.record(stream)
+                sync_all()
+            total_ms, clock_summary = e0.elapsed_time(e1), clocks.summary()
+        else:
+            # One graph of G launches (a multiple of the copy count, so the
+            # rotation runs on across replays), replayed until >= steps.
+            bufs = [(q, k, v, o, lse)] + [
+                (q.clone(), k.clone(), v.clone(), torch.empty_like(o), torch.empty_like(lse))
+                for _ in range(copies - 1)]
+            G = copies * math.ceil(min(steps, 512) / copies)
+            R = math.ceil(steps / G)
+            steps = G * R
+
+            def launch(i):
+                a = bufs[i % copies]
+                fa.fa_fwd(a[0], a[1], a[2], causal=True, out=a[3], lse=a[4], stream=stream,
+                          schedule=sched)
+
+            total_ms, clock_summary = time_graph(launch, G, R, stream, 0, sync_all)
+            del bufs
+        ms = total_ms / steps
         st, word = fa.device_status(stream.cuda_stream)
         if st != fa.FA_OK:
             raise SystemExit(f"kernel status {fa.status_string(st)} {word:#x}")
@@ -660,8 +794,10 @@ def run_sweep(args):
                           "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
                           "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
                           "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                                     "causal": True, "schedule": args.schedule},
-                          "pct_of_peak": 100.0 * value / peak, "peak_source": peak_src}),
+                                     "causal": True, "schedule": sched,
+                                     "l2": l2_note(w.algorithmic_bytes, copies)},
+                          "pct_of_peak": 100.0 * value / peak, "peak_source": peak_src,
+                          "gpu_launches": steps, "clocks": clock_summary}),
               flush=True)
     return 0
 
@@ -677,9 +813,10 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target length of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--schedule", choices=["static", "dynamic"], default="dynamic",
-                    help="work distribution: fa_fwd_dynamic (default; measured 3-5 %% faster "
-                         "on the long causal workloads) or fa_fwd (static)")
+    ap.add_argument("--schedule", choices=["auto", "static", "dynamic"], default="auto",
+                    help="work distribution: fa_fwd_dynamic, fa_fwd (static), or auto (default: "
+                         "dynamic from 4 units of 256 rows per SM, where it measured 2-5 %% faster "
+                         "on long causal workloads; static below, where it saves a few us)")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode-shaped path (HBM-bound) instead of the headline line")
     ap.add_argument("--fp8", action="store_true",

@@ -14,6 +14,6 @@ from ._binding import (  # noqa: F401
     fa_fwd, fa_fwd_raw, fa_fwd_strided_raw, fa_fwd_dynamic_raw, fa_fwd_dynamic_noalloc_raw,
     fa_fwd_debug_raw, device_status, bwd_workspace_bytes, fa_bwd, fa_bwd_raw, fa_bwd_strided_raw, fa_bwd_debug_raw,
     fp8_workspace_bytes, fa_fwd_fp8, fa_fwd_fp8_raw, host_workspace_bytes, fa_fwd_host,
-    fa_fwd_host_raw,
+    fa_fwd_host_raw, resolve_schedule,
 )
 from .autograd import attention  # noqa: F401,E402

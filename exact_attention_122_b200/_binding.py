@@ -415,8 +415,27 @@ def device_status(stream_ptr: int = 0):
     return st, word.value
 
 
+UNIT_ROWS = 256                        # query rows per work unit of the forward kernel
+AUTO_DYNAMIC_UNITS_PER_SM = 4          # "auto": the dynamic schedule from 4 units per SM
+
+
+def resolve_schedule(schedule: str, B: int, H: int, N: int, sm_count: int) -> str:
+    """The schedule fa_fwd uses: "static" or "dynamic" as given; "auto" picks
+    the dynamic schedule from AUTO_DYNAMIC_UNITS_PER_SM units of work per SM
+    (B*H*ceil(N/256) units), the static one below.  Both give identical
+    results; measured on B200, the dynamic schedule's counter reset and
+    claims cost a few microseconds per launch, which only its better
+    balance of long causal problems repays."""
+    if schedule not in ("auto", "static", "dynamic"):
+        raise ValueError("schedule must be 'auto', 'static' or 'dynamic'")
+    if schedule != "auto":
+        return schedule
+    units = B * H * ((N + UNIT_ROWS - 1) // UNIT_ROWS)
+    return "dynamic" if units >= AUTO_DYNAMIC_UNITS_PER_SM * sm_count else "static"
+
+
 def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-           stream=None, schedule: str = "static", workspace=None):
+           stream=None, schedule: str = "auto", workspace=None):
     """O, LSE = exact attention forward of bf16 (B, H, N, d) CUDA tensors.
 
     q, k, v and ``out`` may be strided views (for example a (B, N, H, d)
@@ -424,9 +443,10 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, 
     contiguous; ``out`` (bf16) is allocated contiguous when not given and
     ``lse`` (float32, contiguous (B, H, N)) likewise.  Runs asynchronously on
     ``stream`` (default: the current torch stream of q's device).
-    ``schedule="dynamic"`` uses fa_fwd_dynamic with ``workspace`` (a device
-    tensor of at least DYNAMIC_WORKSPACE_BYTES bytes; one cached per stream
-    when not given).
+    ``schedule="static"`` calls fa_fwd / fa_fwd_strided; ``"dynamic"`` calls
+    fa_fwd_dynamic with ``workspace`` (a device tensor of at least
+    DYNAMIC_WORKSPACE_BYTES bytes; one cached per stream when not given);
+    ``"auto"`` (default) picks one by problem size (resolve_schedule).
     """
     import torch
 
@@ -447,8 +467,8 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, 
         raise ValueError("out must be a bf16 CUDA tensor shaped like q with a contiguous last dimension")
     if not (lse.is_cuda and lse.dtype == torch.float32 and tuple(lse.shape) == (B, H, N) and lse.is_contiguous()):
         raise ValueError("lse must be a contiguous float32 CUDA tensor of shape (B, H, N)")
-    if schedule not in ("static", "dynamic"):
-        raise ValueError("schedule must be 'static' or 'dynamic'")
+    schedule = resolve_schedule(schedule, B, H, N,
+                                torch.cuda.get_device_properties(q.device).multi_processor_count)
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
         contiguous = all(t.is_contiguous() for t in (q, k, v, out))

@@ -107,8 +107,11 @@ fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, f
  *
  * The persistent CTAs claim 256-row units of work from a counter in
  * `workspace` (longest causal rows first, heads grouped for L2 reuse)
- * instead of following a fixed assignment, which balances the CTAs on
- * shapes with few units per SM.  The result is identical to fa_fwd.  The
+ * instead of following a fixed assignment.  This balances long causal
+ * problems better (measured on B200: 2-5 % faster from about 1000 units),
+ * while on small ones (under about 4 units per SM) the counter's reset and
+ * claims cost a few microseconds, so fa_fwd is faster there.  The result is
+ * identical to fa_fwd.  The
  * parallel split over the sequence is the one of the page "FlashAttention:
  * The GPU Memory Hack That Changed Everything", "FlashAttention-2: Even
  * Faster".

@@ -116,3 +116,45 @@ def test_single_process_max_is_identity():
 def test_cli_rejects_short_warmup():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_l2_rotation_plan():
+    """Steps that move less than twice the 126 MB L2 cycle through copies of
+    their buffers: enough that twice the L2 streams between two uses of one
+    copy, at most one copy per launch; big steps use one set of buffers."""
+    L2 = 126 * 1000 * 1000
+    assert bench.rotation_copies(synth.workload(4).algorithmic_bytes, 300) == 1
+    assert bench.rotation_copies(synth.workload(5).algorithmic_bytes, 10) == 1
+    for idx in (1, 2, 3):
+        b = synth.workload(idx).algorithmic_bytes
+        c = bench.rotation_copies(b, 100000)
+        assert c >= 2 and (c - 1) * b >= 2 * L2 and (c - 2) * b < 2 * L2
+        assert bench.rotation_copies(b, 4) == 4       # capped by the launch count
+    assert bench.rotation_copies(2 * L2, 5) == 1
+    assert bench.rotation_copies(2 * L2 - 1, 5) == 3
+    assert "no flush" in bench.l2_note(600_000_000, 1)
+    assert "flushed" in bench.l2_note(25_000_000, 11)
+    with pytest.raises(SystemExit):
+        bench.require_beyond_l2(30_000_000, 20, "--fp8")
+    bench.require_beyond_l2(600_000_000, 20, "--fp8")
+    assert bench.fwd_kernel_name(128) == "fa_fwd_kernel<128,4>"
+    assert bench.fwd_kernel_name(64) == "fa_fwd_kernel<64,8>"
+
+
+def test_auto_schedule_resolution():
+    """"auto" picks the dynamic schedule from 4 units of 256 rows per SM."""
+    from exact_attention_122_b200 import resolve_schedule
+
+    assert resolve_schedule("auto", 2, 32, 8192, 148) == "dynamic"     # 2048 units
+    assert resolve_schedule("auto", 1, 32, 8192, 148) == "dynamic"     # 1024
+    assert resolve_schedule("auto", 1, 32, 4096, 148) == "static"      # 512 < 592
+    assert resolve_schedule("auto", 8, 12, 1024, 148) == "static"      # 384
+    assert resolve_schedule("auto", 1, 37, 4096, 148) == "dynamic"     # 592 = 4 x 148
+    assert resolve_schedule("auto", 1, 37, 4095, 148) == "dynamic"     # ceil(4095/256) = 16
+    assert resolve_schedule("auto", 1, 37, 3840, 148) == "static"      # 555
+    for s in ("static", "dynamic"):
+        assert resolve_schedule(s, 1, 1, 1, 148) == s
+    with pytest.raises(ValueError):
+        resolve_schedule("fast", 1, 1, 1, 148)
+    assert bench.bench_schedule("auto", synth.workload(4)) == "dynamic"
+    assert bench.bench_schedule("auto", synth.workload(2)) == "static"
