@@ -20,7 +20,7 @@
 
 namespace {
 
-constexpr int kMaxDevices = 64;
+constexpr int kMaxDevices = 64;   // current_device() accepts indices below this
 constexpr int kSlots = 2;
 constexpr long long kTargetChunks = 16;
 constexpr long long kUnitRows = 256;   // rows per work unit of the forward kernel

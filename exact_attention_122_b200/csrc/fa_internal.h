@@ -12,7 +12,9 @@ void set_last_cuda_error(int e);
 
 // Current device, checked once per device: FA_OK and its index and SM count
 // when it is an sm_100 device and the tensor-map encoder is available;
-// FA_ERR_NO_DEVICE or FA_ERR_UNSUPPORTED otherwise.
+// FA_ERR_NO_DEVICE or FA_ERR_UNSUPPORTED otherwise.  Device indices of 64
+// and above are refused (FA_ERR_NO_DEVICE), so per-device tables of 64
+// entries are safe to index with the returned index.
 int current_device(int* dev, int* sm_count);
 
 // 4-D bf16 tensor map over (d, N, H, B) with element strides (batch, head,
