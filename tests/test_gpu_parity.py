@@ -393,3 +393,38 @@ def test_decode_matches_square_last_rows(fa, Nq):
     torch.cuda.synchronize()
     assert float((o_dec.float() - o_sq[:, :, N - Nq:].float()).abs().max()) <= TOL_MAX
     assert float((l_dec - l_sq[:, :, N - Nq:]).abs().max()) <= TOL_LSE
+
+
+def test_decode_full_size_sampled(fa):
+    """decode_32k (B=16, H=32, one query against 32768 keys, d=128) in the
+    launch configuration `bench.py --decode` times: automatic split count and
+    a caller workspace.  Every output is finite; sampled (batch, head) rows
+    are compared with the oracle computed row by row."""
+    w = synth.DECODE_WORKLOAD
+    q, k, v = synth.draw_decode_qkv(w.B, w.H, w.Nq, w.Nk, w.d, w.seed)
+    qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
+    ws = torch.empty(fa.decode_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d), dtype=torch.uint8,
+                     device="cuda:0")
+    o, lse = fa.fa_fwd_decode(qd, kd, vd, causal=w.causal, workspace=ws)
+    torch.cuda.synchronize()
+    st, word = fa.device_status()
+    assert st == fa.FA_OK, f"device status {fa.status_string(st)} {word:#x}"
+    assert bool(torch.isfinite(o).all()) and bool(torch.isfinite(lse).all())
+    BH = w.B * w.H
+    q3, k3, v3 = q.view(BH, w.Nq, w.d), k.view(BH, w.Nk, w.d), v.view(BH, w.Nk, w.d)
+    o3 = o.view(BH, w.Nq, w.d).float().cpu().numpy()
+    l3 = lse.view(BH, w.Nq).cpu().numpy()
+    rng = np.random.default_rng(1240)
+    heads = sorted({0, BH - 1} | {int(x) for x in rng.integers(0, BH, size=14)})
+    rows = np.arange(w.Nq)
+    diffs, lse_err = [], 0.0
+    for bh in heads:
+        qb, kb, vb = (oracle.exact_attention._as_f64(t[bh]) for t in (q3, k3, v3))
+        O_ref, L_ref = oracle.attention_rows_fp64(qb, kb, vb, rows, w.causal, w.scale,
+                                                  key_offset=w.Nk - w.Nq)
+        diffs.append(np.abs(o3[bh] - O_ref))
+        lse_err = max(lse_err, float(np.abs(l3[bh] - L_ref).max()))
+    d = np.concatenate(diffs)
+    assert float(d.max()) <= TOL_MAX, float(d.max())
+    assert float(np.sqrt(np.mean(d * d))) <= TOL_RMS
+    assert lse_err <= TOL_LSE, lse_err
