@@ -808,7 +808,7 @@ def run_sweep(args):
                           "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
                           "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                                      "causal": True, "schedule": sched,
-                                     "l2": l2_note(w.algorithmic_bytes, copies, warm)},
+                                     "l2": l2_note(w.algorithmic_bytes, copies)},
                           "pct_of_peak": 100.0 * value / peak, "peak_source": peak_src,
                           "gpu_launches": steps, "clocks": clock_summary}),
               flush=True)

@@ -89,8 +89,20 @@ constexpr float RESCALE_LOG2 = 8.0f;
 #ifndef FA_POLY_COLS
 #define FA_POLY_COLS 0
 #endif
+#ifndef FA_MAX3
+#define FA_MAX3 0
+#endif
 constexpr int POLY_COLS = FA_POLY_COLS;
 static_assert(POLY_COLS >= 0 && POLY_COLS <= 32 && POLY_COLS % 2 == 0, "poly columns");
+
+// P is handed to the MMA thread in P_CHUNKS pieces of BN / P_CHUNKS keys, each
+// with its own barrier, so the P V products of a tile's first keys run on the
+// tensor core while the exponentials of its last keys are still being taken.
+#ifndef FA_PCHUNK
+#define FA_PCHUNK 1
+#endif
+constexpr int P_CHUNKS = FA_PCHUNK ? 4 : 1;
+constexpr int P_CHUNK_KEYS = BN / P_CHUNKS;
 
 enum : uint32_t {
     ROLE_SOFTMAX = 1u, ROLE_MMA = 2u, ROLE_PRODUCER = 3u, ROLE_DRAIN = 4u
@@ -120,13 +132,13 @@ struct Layout {
     static constexpr int B_Q_FULL = 2 * NS;
     static constexpr int B_Q_EMPTY = 2 * NS + 1;
     static constexpr int B_S_FULL = 2 * NS + 2;      // [2]
-    static constexpr int B_P_FULL = 2 * NS + 4;      // [2]
-    static constexpr int B_O_FULL = 2 * NS + 6;      // [2]
-    static constexpr int B_O_EMPTY = 2 * NS + 8;     // [2]
-    static constexpr int B_DRAIN = 2 * NS + 10;
-    static constexpr int B_UFULL = 2 * NS + 11;      // [2] unit queue (dynamic schedule)
-    static constexpr int B_UEMPTY = 2 * NS + 13;     // [2]
-    static constexpr int NUM_BARS = 2 * NS + 15;
+    static constexpr int B_P_FULL = 2 * NS + 4;      // [2][P_CHUNKS]
+    static constexpr int B_O_FULL = B_P_FULL + 2 * P_CHUNKS;   // [2]
+    static constexpr int B_O_EMPTY = B_O_FULL + 2;   // [2]
+    static constexpr int B_DRAIN = B_O_EMPTY + 2;
+    static constexpr int B_UFULL = B_DRAIN + 1;      // [2] unit queue (dynamic schedule)
+    static constexpr int B_UEMPTY = B_UFULL + 2;     // [2]
+    static constexpr int NUM_BARS = B_UEMPTY + 2;
     // tmem base, abort flag, zero flag, spare, unit queue slots [2]
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int OFF_UNIT = OFF_MISC + 16;
@@ -171,62 +183,111 @@ __device__ __forceinline__ void cta_sync() {
     asm volatile("bar.sync 0, %0;" ::"n"(NUM_THREADS) : "memory");
 }
 
-// Software 2^x on the FMA pipe, used for part of each score row so the
-// MUFU unit (ex2) is not the only source of exponentials.  Method:
-// Cody-Waite range reduction x = n + f with n = rint(x) (the 1.5 * 2^23
-// rounding constant), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
+// Software 2^x on the FMA pipe for a packed pair, used for part of each
+// score row so the MUFU unit (ex2) is not the only source of exponentials.
+// Method: Cody-Waite range reduction x = n + f with n = rint(x) (the
+// 1.5 * 2^23 shifter), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
 // coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
 // exchange; csrc/gen_exp2_poly.py reproduces them, max relative error
 // 7.5e-5, below the 2^-9 rounding of the bf16 P it feeds); 2^n is added to
-// the exponent field.  Valid for x in [-126, 64]; inputs below -126 are
-// clamped (results below 2^-125 are meaningless there, so the kernel only
-// uses it on tiles without masked scores).
+// the exponent field with one integer multiply-add per value (the shifter's
+// own bits vanish: they sit above bit 8 of t).  The floating-point steps run
+// as f32x2 pairs.  Valid for x in [-126, 64]; inputs below -126 are clamped
+// (results below 2^-125 are meaningless there, so the kernel only uses it on
+// tiles without masked scores).
 constexpr float EXP2_C0 = 9.999280572e-01f;
 constexpr float EXP2_C1 = 6.932609677e-01f;
 constexpr float EXP2_C2 = 2.426111251e-01f;
 constexpr float EXP2_C3 = 5.517166853e-02f;
 
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -126.0f);
-    const float t = x + 12582912.0f;            // 1.5 * 2^23: t's low bits hold rint(x)
-    const float n = t - 12582912.0f;
-    const float f = x - n;
-    const float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, EXP2_C0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& y0, float& y1) {
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+    const uint64_t sh = f2_pack(12582912.0f, 12582912.0f);         // 1.5 * 2^23
+    const uint64_t t = f2_add(xc, sh);           // low mantissa bits of t hold rint(x)
+    const uint64_t f = f2_sub(xc, f2_sub(t, sh));
+    uint64_t p = f2_fma(f2_pack(EXP2_C3, EXP2_C3), f, f2_pack(EXP2_C2, EXP2_C2));
+    p = f2_fma(p, f, f2_pack(EXP2_C1, EXP2_C1));
+    p = f2_fma(p, f, f2_pack(EXP2_C0, EXP2_C0));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    y0 = __uint_as_float(__float_as_uint(p0) + __float_as_uint(t0) * (1u << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + __float_as_uint(t1) * (1u << 23));
 }
 
 // ---------------------------------------------------------------------------
-// Work decomposition: units of 256 query rows of one (batch, head).
-// Units are ordered in groups of `hg` heads (sized on the host so a group's
-// K and V stay resident in L2 while the CTAs working on it stream them);
-// inside a group the order is by row block, the longest causal rows first.
-// CTA b takes sequence indices in boustrophedon order (b, 2S-1-b, 2S+b, ...)
-// so long and short units pair up across CTAs.
+// Work decomposition: units of 256 query rows of one (batch, head), named by
+// the id c = bh * nq2 + qb2 (qb2: the unit's 256-row block).
+//
+// Both schedules walk heads in groups of `hg` (sized on the host so a
+// group's K and V stay resident in L2 while the CTAs working on it stream
+// them).
+//  * Sequence order (the dynamic schedule's claim order, and the static
+//    "snake" assignment): inside a group, by row block, the longest causal
+//    rows first; static CTA b takes sequence indices in boustrophedon order
+//    (b, 2S-1-b, 2S+b, ...) so long and short units pair up across CTAs.
+//  * Paired static assignment (causal): the row blocks q and nq2-1-q of one
+//    head form a pair whose K/V tile count hardly depends on q, so dealing
+//    pairs round-robin (CTA b takes pairs b, b+S, b+2S, ..., the long unit of
+//    each pair first) balances the CTAs to within one pair whatever the group
+//    size.  With an odd nq2 the middle row block is a pair of one unit.
 // ---------------------------------------------------------------------------
 struct Unit {
     int bh, r0, nb0, nb1;  // first row, K/V tile counts of sub-tiles 0 and 1
 };
 
+constexpr int UNIT_END = -1;   // no more units for this CTA
+constexpr int UNIT_SKIP = -2;  // static paired schedule: empty second half of a pair
+
 __device__ __forceinline__ int unit_index(int k, int cta, int ctas) {
     return k * ctas + ((k & 1) ? (ctas - 1 - cta) : cta);
 }
 
-// N_q query rows and N_k keys per (batch, head); with causal masking query i
-// may see key j iff j <= i + N_k - N_q (the queries are the last N_q
-// positions), so a sub-tile's last row r sees keys up to r + N_k - N_q.
-__device__ __forceinline__ Unit decode_unit(int i, int BH, int Nq, int Nk, int causal, int hg) {
-    const int nq2 = (Nq + UNIT_ROWS - 1) / UNIT_ROWS;
-    const int nkb = (Nk + BN - 1) / BN;
-    const int off = Nk - Nq;
+// Sequence index i (grouped, longest first) -> unit id.
+__device__ __forceinline__ int seq_to_unit(int i, int BH, int nq2, int causal, int hg) {
     const int per_group = hg * nq2;
     const int g = i / per_group;
     const int r = i - g * per_group;
     const int gh = min(hg, BH - g * hg);       // heads in this group
     const int level = r / gh;
+    const int bh = g * hg + (r - level * gh);
+    return bh * nq2 + (causal ? (nq2 - 1 - level) : level);
+}
+
+// The kq-th unit of CTA `cta` under the static schedule: a unit id,
+// UNIT_END, or UNIT_SKIP (move on to kq + 1).
+__device__ __forceinline__ int static_unit(int kq, int cta, int ctas, int BH, int nq2, int causal,
+                                           int hg, int paired) {
+    if (!paired) {
+        const int i = unit_index(kq, cta, ctas);
+        return i < BH * nq2 ? seq_to_unit(i, BH, nq2, causal, hg) : UNIT_END;
+    }
+    const int npl = (nq2 + 1) / 2;             // pairs per head
+    const int p = (kq >> 1) * ctas + cta;
+    if (p >= BH * npl) return UNIT_END;
+    const int per_group = hg * npl;
+    const int g = p / per_group;
+    const int r = p - g * per_group;
+    const int gh = min(hg, BH - g * hg);
+    const int pl = r / gh;
+    const int bh = g * hg + (r - pl * gh);
+    const int q_long = nq2 - 1 - pl;
+    if (kq & 1) return pl == q_long ? UNIT_SKIP : bh * nq2 + pl;
+    return bh * nq2 + q_long;
+}
+
+// N_q query rows and N_k keys per (batch, head); with causal masking query i
+// may see key j iff j <= i + N_k - N_q (the queries are the last N_q
+// positions), so a sub-tile's last row r sees keys up to r + N_k - N_q.
+__device__ __forceinline__ Unit decode_unit(int c, int Nq, int Nk, int causal) {
+    const int nq2 = (Nq + UNIT_ROWS - 1) / UNIT_ROWS;
+    const int nkb = (Nk + BN - 1) / BN;
+    const int off = Nk - Nq;
     Unit w;
-    w.bh = g * hg + (r - level * gh);
-    const int qb2 = causal ? (nq2 - 1 - level) : level;
-    w.r0 = qb2 * UNIT_ROWS;
+    w.bh = c / nq2;
+    w.r0 = (c - w.bh * nq2) * UNIT_ROWS;
     if (causal) {
         w.nb0 = min((w.r0 + BM - 1 + off) / BN + 1, nkb);
         w.nb1 = min((w.r0 + 2 * BM - 1 + off) / BN + 1, nkb);
@@ -254,21 +315,28 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint6
     }
 }
 
-// O += P V for one sub-tile: A = P from TMEM (8 columns per step: 16 keys
-// as bf16 pairs, or 32 keys as FP8 quads).  bf16: B = V MN-major, 16 key
-// rows of 128 bytes per step.  FP8: B = V^T K-major (d rows of 128 keys), a
-// step is 32 bytes inside the swizzled rows.
+// O += P V for one sub-tile over keys [c * P_CHUNK_KEYS, (c + 1) *
+// P_CHUNK_KEYS) of the tile: A = P from TMEM (8 columns per step: 16 keys as
+// bf16 pairs, or 32 keys as FP8 quads).  bf16: B = V MN-major, 16 key rows of
+// 128 bytes per step.  FP8: B = V^T K-major (d rows of 128 keys), a step is
+// 32 bytes inside the swizzled rows.  `first`: the tile's first chunk of a
+// unit's first tile overwrites O instead of accumulating.
 template <bool F8>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc,
-                                         uint32_t idesc, bool first) {
+                                         uint32_t idesc, int c, bool first) {
     if constexpr (F8) {
+        constexpr int STEPS = P_CHUNK_KEYS / 32;
 #pragma unroll
-        for (int kk = 0; kk < BN / 32; ++kk)
+        for (int i = 0; i < STEPS; ++i) {
+            const int kk = c * STEPS + i;
             mma_ts_f8(o_tmem, p_tmem + kk * 8, desc_add(v_desc, uint32_t((kk * 32) >> 4)), idesc,
                       (first && kk == 0) ? 0u : 1u);
+        }
     } else {
+        constexpr int STEPS = P_CHUNK_KEYS / 16;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
+        for (int i = 0; i < STEPS; ++i) {
+            const int kk = c * STEPS + i;
             const uint32_t off = uint32_t((kk * 16 * 128) >> 4);
             mma_ts(o_tmem, p_tmem + kk * 8, desc_add(v_desc, off), idesc,
                    (first && kk == 0) ? 0u : 1u);
@@ -276,14 +344,32 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
     }
 }
 
+// p rounded the way exp_row_to_p rounds P for the P V product: bf16 (nearest
+// even) or, with F8, FP8 E4M3 (nearest even, saturating).
+template <bool F8>
+__device__ __forceinline__ float round_as_p(float p) {
+    if constexpr (F8) {
+        uint16_t q8;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(q8) : "f"(0.0f), "f"(p));
+        uint32_t h2;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(q8));
+        return __half2float(__ushort_as_half(uint16_t(h2 & 0xFFFFu)));
+    } else {
+        return __bfloat162float(__float2bfloat16_rn(p));
+    }
+}
+
 // P = 2^(s * scale_log2 - m) for one score row held in registers, written
 // to TMEM over the row's first columns: bf16 pairs (64 columns) or, with F8,
 // FP8 E4M3 quads (32 columns).  The row sum (of the unrounded fp32 P) goes to
 // four packed partial accumulators.  The first NPOLY columns of every
-// 32-column chunk use exp2_poly, the rest MUFU ex2.
+// 32-column chunk use exp2_poly_x2, the rest MUFU ex2.  Each chunk of
+// P_CHUNK_KEYS keys is published on its barrier (p_bar + 8 c) once its TMEM
+// stores have completed.
 template <int NPOLY, bool F8 = false>
 __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_log2, float neg_m,
-                                             uint64_t (&acc)[4], uint32_t tS) {
+                                             uint64_t (&acc)[4], uint32_t tS, uint32_t p_bar) {
+    static_assert(P_CHUNK_KEYS % 32 == 0, "P chunks are whole 32-key groups");
     const uint64_t c2 = f2_pack(scale_log2, scale_log2);
     const uint64_t m2 = f2_pack(neg_m, neg_m);
     uint64_t pf_prev = 0;                        // F8: the previous pair of P values
@@ -296,8 +382,7 @@ __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_l
             f2_unpack(f2_fma(f2_pack(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), c2, m2), x0, x1);
             float p0, p1;
             if (2 * i < NPOLY) {
-                p0 = exp2_poly(x0);
-                p1 = exp2_poly(x1);
+                exp2_poly_x2(f2_pack(x0, x1), p0, p1);
             } else {
                 p0 = ex2(x0);
                 p1 = ex2(x1);
@@ -320,6 +405,11 @@ __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_l
             tmem_st8(tS + c * 8, pk);            // P (FP8) over S columns [0, 32)
         else
             tmem_st16(tS + c * 16, pk);          // P (bf16) over S columns [0, 64)
+        if ((c + 1) % (P_CHUNK_KEYS / 32) == 0) {
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(p_bar + 8u * uint32_t(c / (P_CHUNK_KEYS / 32)));
+        }
     }
 }
 
@@ -335,7 +425,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ Og,
                   float* __restrict__ LSEg, int BH, int H, int Nq, int Nk, int causal,
                   float scale_log2,
-                  int hg, long long o_sb, long long o_sh, long long o_sn, int* __restrict__ sched,
+                  int hg, int paired, long long o_sb, long long o_sh, long long o_sn,
+                  int* __restrict__ sched,
                   unsigned long long watchdog_ns, int inject, float o_scale) {
     using L = Layout<D, NS, F8>;
     extern __shared__ uint8_t smem_raw[];
@@ -361,15 +452,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int koff = Nk - Nq;                  // causal: key j allowed for row i iff j <= i + koff
     const Watchdog wd_in{abort_flag, watchdog_ns};
     // Unit queue.  Static schedule (sched == nullptr): every role walks the
-    // same boustrophedon sequence.  Dynamic schedule: the producer claims
-    // sequence indices from the global counter *sched and publishes them in
-    // two shared-memory slots (full: producer; empty: MMA thread and every
-    // softmax thread); -1 ends the CTA's work.
-    auto next_unit_consumer = [&](int kq, bool& ok_out, uint32_t role) -> int {
-        if (!sched) {
-            const int u = unit_index(kq, blockIdx.x, gridDim.x);
-            return u < num_units ? u : -1;
-        }
+    // same assignment (static_unit), skipping the same empty entries.
+    // Dynamic schedule: the producer claims sequence indices from the global
+    // counter *sched and publishes their unit ids in two shared-memory slots
+    // (full: producer; empty: MMA thread and every softmax thread); -1 ends
+    // the CTA's work.
+    auto next_static = [&](int& kq) -> int {
+        int u;
+        while ((u = static_unit(kq, blockIdx.x, gridDim.x, BH, nq2, causal, hg, paired)) ==
+               UNIT_SKIP)
+            ++kq;
+        return u;
+    };
+    auto next_unit_consumer = [&](int& kq, bool& ok_out, uint32_t role) -> int {
+        if (!sched) return next_static(kq);
         const int slot = kq & 1;
         bool got = wait_phase(bar(L::B_UFULL + slot), uint32_t(kq >> 1) & 1u, wd_in, role, 0);
         if (role == ROLE_SOFTMAX) got = __all_sync(0xffffffffu, got);
@@ -391,7 +487,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_init(bar(L::B_Q_EMPTY), 1);
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(L::B_S_FULL + t), 1);
-            mbar_init(bar(L::B_P_FULL + t), BM);
+            for (int c = 0; c < P_CHUNKS; ++c) mbar_init(bar(L::B_P_FULL + t * P_CHUNKS + c), BM);
             mbar_init(bar(L::B_O_FULL + t), 1);
             mbar_init(bar(L::B_O_EMPTY + t), BM);
         }
@@ -441,15 +537,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         break;
                     }
                     u = atomicAdd(sched, 1);
-                    if (u >= num_units) u = -1;
+                    u = u < num_units ? seq_to_unit(u, BH, nq2, causal, hg) : UNIT_END;
                     unit_slot[slot] = u;
                     mbar_arrive(bar(L::B_UFULL + slot));
                 } else {
-                    u = unit_index(kq, blockIdx.x, gridDim.x);
-                    if (u >= num_units) u = -1;
+                    u = next_static(kq);
                 }
                 if (u < 0) break;
-                const Unit w = decode_unit(u, BH, Nq, Nk, causal, hg);
+                const Unit w = decode_unit(u, Nq, Nk, causal);
                 const int wb = w.bh / H, wh = w.bh - (w.bh / H) * H;   // batch, head
                 if (!wait_phase(bar(L::B_Q_EMPTY), (units & 1u) ^ 1u, wd, ROLE_PRODUCER, u)) {
                     ok = false;
@@ -531,10 +626,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t stage_step = uint32_t(L::KV_BYTES >> 4);
             const uint32_t tS0 = tmem + L::TM_S0, tS1 = tmem + L::TM_S1;
             const uint32_t tO0 = tmem + L::TM_O0, tO1 = tmem + L::TM_O1;
+            // O_t += P_t V for one tile, each chunk of keys as soon as the
+            // softmax warpgroup has published its part of P_t.
+            auto pv_chunks = [&](int t, uint32_t pcnt, uint32_t tO, uint32_t tS, uint64_t v_desc,
+                                 bool first, int u) -> bool {
+#pragma unroll
+                for (int c = 0; c < P_CHUNKS; ++c) {
+                    if (!wait_phase(bar(L::B_P_FULL + t * P_CHUNKS + c), pcnt & 1u, wd, ROLE_MMA, u))
+                        return false;
+                    tc_fence_after();
+                    issue_pv<F8>(tO, tS, v_desc, ID_PV, c, first);
+                }
+                return true;
+            };
             for (int kq = 0; ok; ++kq, ++units) {
                 const int u = next_unit_consumer(kq, ok, ROLE_MMA);
                 if (u < 0) break;
-                const Unit w = decode_unit(u, BH, Nq, Nk, causal, hg);
+                const Unit w = decode_unit(u, Nq, Nk, causal);
                 if (!wait_phase(bar(L::B_Q_FULL), units & 1u, wd, ROLE_MMA, u)) { ok = false; break; }
                 uint32_t sK = cons % NS;
                 if (!wait_phase(bar(L::B_KV_FULL + sK), (cons / NS) & 1u, wd, ROLE_MMA, u)) {
@@ -571,13 +679,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             ok = false;
                             break;
                         }
-                        if (!wait_phase(bar(L::B_P_FULL + 0), pcnt0 & 1u, wd, ROLE_MMA, u)) {
+                        if (!pv_chunks(0, pcnt0, tO0, tS0, desc_add(dv0, sV * stage_step), j == 0, u)) {
                             ok = false;
                             break;
                         }
                         ++pcnt0;
-                        tc_fence_after();
-                        issue_pv<F8>(tO0, tS0, desc_add(dv0, sV * stage_step), ID_PV, j == 0);
                         if (j + 1 < w.nb0) {
                             issue_qk<L::QK_STEPS, L::HALF_BYTES, F8>(tS0, dq0, desc_add(dk0, sK * stage_step), ID_S);
                             tc_commit(bar(L::B_S_FULL + 0));
@@ -588,13 +694,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                         break;
                     }
-                    if (!wait_phase(bar(L::B_P_FULL + 1), pcnt1 & 1u, wd, ROLE_MMA, u)) {
+                    if (!pv_chunks(1, pcnt1, tO1, tS1, desc_add(dv0, sV * stage_step), j == 0, u)) {
                         ok = false;
                         break;
                     }
                     ++pcnt1;
-                    tc_fence_after();
-                    issue_pv<F8>(tO1, tS1, desc_add(dv0, sV * stage_step), ID_PV, j == 0);
                     if (next) {
                         issue_qk<L::QK_STEPS, L::HALF_BYTES, F8>(tS1, dq1, desc_add(dk0, sK * stage_step), ID_S);
                         tc_commit(bar(L::B_S_FULL + 1));
@@ -639,12 +743,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kq = 0; ok; ++kq) {
             const int u = next_unit_consumer(kq, ok, ROLE_SOFTMAX);
             if (u < 0) break;
-            const Unit w = decode_unit(u, BH, Nq, Nk, causal, hg);
+            const Unit w = decode_unit(u, Nq, Nk, causal);
             const int a = w.r0 + t * BM;             // first row of this sub-tile
             const int row = a + wr;
             const int nb = t == 0 ? w.nb0 : w.nb1;
             float m = -INFINITY;                     // running max, log2 units
             float l = 0.f;                           // running sum of exponentials
+            float lc = 0.f;                          // rounding correction of l for O
             for (int j = 0; j < nb; ++j) {
                 bool got = wait_phase(bar(L::B_S_FULL + t), scnt & 1u, wd, ROLE_SOFTMAX, u);
                 ++scnt;
@@ -671,17 +776,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         s[c] = bad ? -INFINITY : s[c];
                     }
                 }
-                // Row max: eight independent chains, then a tree.  (The
-                // three-input max.f32 form measured inexact here: it broke the
-                // bit-exact causal row 0 of the parity tests.)
+                // Row max: eight independent chains, then a tree.
                 float mx8[8];
+#if FA_MAX3
+                // three-input max: about half the instructions of two-input
+                // chains.  Chain i takes columns i, i+8, ..., i+120.
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx8[i] = fmax3(s[i], s[8 + i], s[16 + i]);
+#pragma unroll
+                for (int c = 24; c < BN - 8; c += 16) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[c + i], s[c + 8 + i]);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], s[BN - 8 + i]);
+                const float s_top = fmaxf(fmax3(fmax3(mx8[0], mx8[1], mx8[2]),
+                                                fmax3(mx8[3], mx8[4], mx8[5]), mx8[6]),
+                                          mx8[7]);
+#else
 #pragma unroll
                 for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
                 for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-                const float m_blk =
+                const float s_top =
                     fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+#endif
+                const float m_blk = s_top * scale_log2;
                 // Lazy rescale (first tile: m = -inf, so every lane moves).
                 if (__any_sync(0xffffffffu, m_blk > m + RESCALE_LOG2)) {
                     const float m_new = fmaxf(m, m_blk);
@@ -700,16 +821,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         }
                     }
                     l *= alpha;
+                    lc *= alpha;
                     m = m_new;
                 }
                 const float neg_m = -m;
+                // The P V product takes P rounded to its operand type, while
+                // l sums the unrounded P.  O is normalised by l + lc, lc
+                // holding the rounding error of each tile's largest P: with a
+                // stale reference m that P is not a power of two, and when it
+                // dominates the row (peaked attention) its rounding then
+                // cancels between O's numerator and normaliser.  The LSE
+                // keeps the unrounded l.
+                {
+                    const float p_top = ex2(fmaf(s_top, scale_log2, neg_m));
+                    lc += round_as_p<F8>(p_top) - p_top;
+                }
                 uint64_t acc[4] = {0, 0, 0, 0};              // four packed (0.f, 0.f)
                 // Tiles without masked scores may use the FMA-pipe 2^x for
                 // part of the row; the choice is warp-uniform, made once.
+                const uint32_t p_bar = bar(L::B_P_FULL + t * P_CHUNKS);
                 if (POLY_COLS > 0 && !(tail || diag))
-                    exp_row_to_p<POLY_COLS, F8>(s, scale_log2, neg_m, acc, tS);
+                    exp_row_to_p<POLY_COLS, F8>(s, scale_log2, neg_m, acc, tS, p_bar);
                 else
-                    exp_row_to_p<0, F8>(s, scale_log2, neg_m, acc, tS);
+                    exp_row_to_p<0, F8>(s, scale_log2, neg_m, acc, tS, p_bar);
                 {
                     float a0, a1, a2, a3, a4, a5, a6, a7;
                     f2_unpack(acc[0], a0, a1);
@@ -718,9 +852,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     f2_unpack(acc[3], a6, a7);
                     l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(L::B_P_FULL + t));
             }
             if (!ok) break;
             // Epilogue: O / l -> bf16 -> global; LSE.
@@ -728,7 +859,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ++ocnt;
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
-            float inv_l = 1.f / l;
+            float inv_l = 1.f / (l + lc);
             if constexpr (F8) inv_l *= o_scale;
             const bool store = row < Nq;
             const int wb = w.bh / H, wh = w.bh - (w.bh / H) * H;     // batch, head
@@ -875,17 +1006,19 @@ int fa_internal::encode_bhnd_map(CUtensorMap* map, const void* base, int d, int 
 
 namespace {
 
-// Heads per scheduling group.  The kernel orders units in groups of `hg`
-// heads (longest causal row blocks first inside a group) and deals them to
-// CTAs in boustrophedon order (decode_unit / unit_index).  Small groups keep
-// the K/V that concurrently running CTAs stream resident in L2; large groups
-// balance the CTAs better.  This replays the kernel's assignment on the host
-// for hg = 1, 2, 4, ..., BH (K/V tiles per unit as the cost) and takes the
-// lowest  (max CTA load / mean CTA load) x (1 + L2 penalty), the penalty
-// growing with the group's K/V bytes: 0 up to 16 MiB, then 3 %, 6 %, 9 % and
-// 12 % past 16, 32, 64 and 128 MiB (calibrated on the 8K and 32K causal
-// workloads, where 2-head groups measured 4-7 % faster than 8- or all-head
-// groups).  Decisions are cached per shape.
+// Static schedule choice: the assignment (snake or paired, see static_unit)
+// and the heads per group.  Small groups keep the K/V that concurrently
+// running CTAs stream resident in L2; with the snake, large groups balance
+// the CTAs better, while the paired assignment balances long causal
+// problems at any group size once every CTA holds several pairs.  This
+// replays the kernel's assignment on the host for both assignments and
+// hg = 1, 2, 4, ..., BH (K/V tiles per unit plus a fixed per-unit overhead
+// as the cost) and takes the lowest (max CTA load / mean CTA load) x
+// (1 + L2 penalty), the penalty growing with the group's K/V bytes: 0 up to
+// 16 MiB, then 3 %, 6 %, 9 % and 12 % past 16, 32, 64 and 128 MiB
+// (calibrated on the 8K and 32K causal workloads, where 2-head snake groups
+// measured 4-7 % faster than 8- or all-head groups).  Decisions are cached
+// per shape.
 struct HgKey {
     long long BH;
     int Nq, Nk, D, causal, grid;
@@ -894,29 +1027,52 @@ struct HgKey {
                grid == o.grid;
     }
 };
+struct StaticPlan {
+    long long hg;
+    int paired;
+};
 std::mutex g_hg_mutex;
 HgKey g_hg_keys[64];
-long long g_hg_vals[64];
+StaticPlan g_hg_vals[64];
 int g_hg_count = 0;
 
-double snake_imbalance(long long BH, int Nq, int Nk, int causal, long long hg, int grid) {
+// Max CTA load over mean CTA load of the static assignment, replayed.
+double static_imbalance(long long BH, int Nq, int Nk, int causal, long long hg, int paired,
+                        int grid) {
     const long long nq2 = (Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
     const long long nkb = (Nk + fa::BN - 1) / fa::BN;
     const long long off = Nk - Nq;
-    const long long units = nq2 * BH;
     std::vector<long long> load(size_t(grid), 0);
-    const long long per_group = hg * nq2;
-    for (long long i = 0; i < units; ++i) {
-        const long long g = i / per_group;
-        const long long r = i - g * per_group;
-        const long long gh = std::min(hg, BH - g * hg);
-        const long long level = r / gh;
-        const long long r0 = (causal ? (nq2 - 1 - level) : level) * fa::UNIT_ROWS;
+    auto cost = [&](long long qb2) {            // K/V tiles of both sub-tiles + overhead
+        const long long r0 = qb2 * fa::UNIT_ROWS;
         const long long nb0 = causal ? std::min((r0 + fa::BM - 1 + off) / fa::BN + 1, nkb) : nkb;
         const long long nb1 =
             causal ? std::min((r0 + 2 * fa::BM - 1 + off) / fa::BN + 1, nkb) : nkb;
-        const long long k = i / grid, c = i - k * grid;
-        load[size_t((k & 1) ? (grid - 1 - c) : c)] += nb0 + nb1 + 2;   // +2: per-unit overhead
+        return nb0 + nb1 + 2;
+    };
+    if (!paired) {
+        const long long units = nq2 * BH;
+        const long long per_group = hg * nq2;
+        for (long long i = 0; i < units; ++i) {
+            const long long g = i / per_group;
+            const long long r = i - g * per_group;
+            const long long gh = std::min(hg, BH - g * hg);
+            const long long level = r / gh;
+            const long long k = i / grid, c = i - k * grid;
+            load[size_t((k & 1) ? (grid - 1 - c) : c)] += cost(causal ? nq2 - 1 - level : level);
+        }
+    } else {
+        // CTA c takes pairs c, c + grid, ... (both units of each pair).
+        const long long npl = (nq2 + 1) / 2;
+        const long long per_group = hg * npl;
+        for (long long p = 0; p < BH * npl; ++p) {
+            const long long g = p / per_group;
+            const long long r = p - g * per_group;
+            const long long gh = std::min(hg, BH - g * hg);
+            const long long pl = r / gh;
+            const long long q_long = nq2 - 1 - pl;
+            load[size_t(p % grid)] += cost(q_long) + (pl == q_long ? 0 : cost(pl));
+        }
     }
     long long mx = 0, sum = 0;
     for (long long x : load) {
@@ -926,7 +1082,7 @@ double snake_imbalance(long long BH, int Nq, int Nk, int causal, long long hg, i
     return double(mx) * grid / double(sum);
 }
 
-long long choose_head_group(long long BH, int Nq, int Nk, int D, int causal, int grid) {
+StaticPlan choose_static_plan(long long BH, int Nq, int Nk, int D, int causal, int grid) {
     const HgKey key{BH, Nq, Nk, D, causal, grid};
     {
         std::lock_guard<std::mutex> lk(g_hg_mutex);
@@ -934,24 +1090,27 @@ long long choose_head_group(long long BH, int Nq, int Nk, int D, int causal, int
             if (g_hg_keys[i] == key) return g_hg_vals[i];
     }
     const long long kv_head_bytes = 2LL * Nk * D * 2;
-    long long best = BH;
+    StaticPlan best{BH, 0};
     double best_cost = 1e30;
     // Bound the replay work for very large problems: beyond ~4M units the
     // assignment statistics no longer depend on hg, so all heads form one group.
     const long long units = ((Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS) * BH;
     if (units <= (4LL << 20)) {
-        for (long long hg = 1;; hg = std::min(hg * 2, BH)) {
-            const double ws = double(hg * kv_head_bytes);
-            const double pen = ws <= 16.0 * (1 << 20) ? 0.0
-                             : ws <= 32.0 * (1 << 20) ? 0.03
-                             : ws <= 64.0 * (1 << 20) ? 0.06
-                             : ws <= 128.0 * (1 << 20) ? 0.09 : 0.12;
-            const double cost = snake_imbalance(BH, Nq, Nk, causal, hg, grid) * (1.0 + pen);
-            if (cost < best_cost - 1e-9) {
-                best_cost = cost;
-                best = hg;
+        for (int paired = 0; paired <= (causal ? 1 : 0); ++paired) {
+            for (long long hg = 1;; hg = std::min(hg * 2, BH)) {
+                const double ws = double(hg * kv_head_bytes);
+                const double pen = ws <= 16.0 * (1 << 20) ? 0.0
+                                 : ws <= 32.0 * (1 << 20) ? 0.03
+                                 : ws <= 64.0 * (1 << 20) ? 0.06
+                                 : ws <= 128.0 * (1 << 20) ? 0.09 : 0.12;
+                const double cost =
+                    static_imbalance(BH, Nq, Nk, causal, hg, paired, grid) * (1.0 + pen);
+                if (cost < best_cost - 1e-9) {
+                    best_cost = cost;
+                    best = StaticPlan{hg, paired};
+                }
+                if (hg == BH) break;
             }
-            if (hg == BH) break;
         }
     }
     std::lock_guard<std::mutex> lk(g_hg_mutex);
@@ -995,12 +1154,18 @@ fa_status launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     // group size; groups then hold about 16 MiB of K/V (all heads when the
     // whole K/V fits in 32 MiB).
     const long long kv_head_bytes = 2LL * Nk * D * L::EB;
-    long long hg = sched ? ((BH * kv_head_bytes <= (32LL << 20)) ? BH : (16LL << 20) / kv_head_bytes)
-                         : choose_head_group(BH, Nq, Nk, D, causal, grid);
+    StaticPlan plan{BH, 0};
+    if (sched)
+        plan.hg = (BH * kv_head_bytes <= (32LL << 20)) ? BH : (16LL << 20) / kv_head_bytes;
+    else
+        plan = choose_static_plan(BH, Nq, Nk, D, causal, grid);
 #ifdef FA_HEAD_GROUP
-    hg = FA_HEAD_GROUP;
+    plan.hg = FA_HEAD_GROUP;
 #endif
-    hg = hg < 1 ? 1 : (hg > BH ? BH : hg);
+#ifdef FA_STATIC_PAIRED
+    plan.paired = causal ? FA_STATIC_PAIRED : 0;
+#endif
+    const long long hg = plan.hg < 1 ? 1 : (plan.hg > BH ? BH : plan.hg);
     if (sched) {
         const cudaError_t me = cudaMemsetAsync(sched, 0, sizeof(int), stream);
         if (me != cudaSuccess) {
@@ -1010,7 +1175,8 @@ fa_status launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     }
     kern<<<grid, fa::NUM_THREADS, L::ALLOC, stream>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o),
                                                      lse, int(BH), H, Nq, Nk, causal, scale_log2,
-                                                     int(hg), ost.b, ost.h, ost.n, sched,
+                                                     int(hg), plan.paired, ost.b, ost.h, ost.n,
+                                                     sched,
                                                      watchdog_ns, inject, o_scale);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
@@ -1218,10 +1384,14 @@ fa_status fa_fwd_dynamic_noalloc(const void* q, const void* k, const void* v, vo
                                  int B, int H, int N, int d, const long long* strides, int causal,
                                  float scale, void* stream) {
     // The scratch holds one 32-bit counter of claimed units: problems with
-    // more units than it may count are refused before anything else.
-    if (B >= 1 && H >= 1 && N >= 1 &&
-        ((long long)N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS * B * H > FA_NOALLOC_MAX_UNITS)
-        return FA_ERR_UNSUPPORTED;
+    // more units than it may count are refused before anything else.  B*H is
+    // bounded first so the unit count cannot overflow.
+    if (B >= 1 && H >= 1 && N >= 1) {
+        const long long bh = (long long)B * H;
+        if (bh > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+        if (((long long)N + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS > FA_NOALLOC_MAX_UNITS / bh)
+            return FA_ERR_UNSUPPORTED;
+    }
     if (FA_DYNAMIC_WORKSPACE_BYTES > sizeof(fa::g_noalloc_scratch)) return FA_ERR_UNSUPPORTED;
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);

@@ -27,8 +27,10 @@
  *    synchronised that stream.
  *  - Arguments are validated before anything is enqueued; an invalid call
  *    returns an error status and has no side effect.
- *  - Calls are thread-safe.  One call per stream at a time may run on a
- *    device; concurrent calls on different streams are independent.
+ *  - Calls are thread-safe.  Calls on different streams compute
+ *    independently (each uses only its own arguments and workspace), with
+ *    one exception: the watchdog status word read by fa_get_device_status
+ *    is one per device, shared by all streams (see there).
  *  - Inputs holding NaN or Inf are not detected; they propagate.
  */
 #ifndef FA_B200_H
@@ -401,6 +403,14 @@ fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, flo
  * FA_ERR_TIMEOUT (a kernel watchdog fired since the last read); *detail, if
  * not NULL, receives the raw word (role and unit of the first timeout).
  * Returns FA_ERR_NO_DEVICE / FA_ERR_LAUNCH if the CUDA calls fail.
+ *
+ * The word is one per device (one for the forward kernels, one for the
+ * backward kernels, reported together), not one per stream or call: a
+ * timeout in a call on any stream is reported to, and cleared by, the next
+ * reader on that device, whichever stream it synchronises.  Only the first
+ * timeout since the last read is kept.  Callers that run several streams
+ * and need to know which call timed out should synchronise all of them
+ * before reading.
  */
 fa_status fa_get_device_status(void* stream, unsigned* detail);
 
