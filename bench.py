@@ -3,8 +3,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one exact-attention forward (one fa_fwd_dynamic launch: the
-"auto" schedule picks it for this size; --schedule static times fa_fwd) over
+A step is one exact-attention forward (one launch of the C entry point fa_fwd:
+the "auto" schedule picks the static schedule for this size; --schedule
+dynamic times fa_fwd_dynamic) over
 one batch of the long-context causal workload (B=2, H=32, N=8192, d=128, bf16, seeded
 N(0,1) inputs), inputs resident in HBM.  FLOPs per step: 4*B*H*N^2*d / 2.
 Prints one JSON line (rank 0).
@@ -828,8 +829,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", choices=["auto", "static", "dynamic"], default="auto",
                     help="work distribution: fa_fwd_dynamic, fa_fwd (static), or auto (default: "
-                         "dynamic from 4 units of 256 rows per SM, where it measured 2-5 %% faster "
-                         "on long causal workloads; static below, where it saves a few us)")
+                         "dynamic from 4 to 12 units of 256 rows per SM, static otherwise)")
     ap.add_argument("--l2-warm", action="store_true",
                     help="time the forward line on one reused set of buffers without an L2 flush "
                          "(graph-replayed): the L2-warm figure for workloads that fit in L2")

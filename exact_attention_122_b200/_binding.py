@@ -416,22 +416,26 @@ def device_status(stream_ptr: int = 0):
 
 
 UNIT_ROWS = 256                        # query rows per work unit of the forward kernel
-AUTO_DYNAMIC_UNITS_PER_SM = 4          # "auto": the dynamic schedule from 4 units per SM
+AUTO_DYNAMIC_UNITS_PER_SM = (4, 12)    # "auto": the dynamic schedule in this units-per-SM band
 
 
 def resolve_schedule(schedule: str, B: int, H: int, N: int, sm_count: int) -> str:
     """The schedule fa_fwd uses: "static" or "dynamic" as given; "auto" picks
-    the dynamic schedule from AUTO_DYNAMIC_UNITS_PER_SM units of work per SM
-    (B*H*ceil(N/256) units), the static one below.  Both give identical
-    results; measured on B200, the dynamic schedule's counter reset and
-    claims cost a few microseconds per launch, which only its better
-    balance of long causal problems repays."""
+    the dynamic schedule when the problem has between 4 and 12 units of work
+    per SM (B*H*ceil(N/256) units), the static one otherwise.  Both give
+    identical results.  Measured on B200: below 4 units per SM the dynamic
+    schedule's counter reset and claims cost a few microseconds per launch;
+    from 12 units per SM the static schedule's paired causal assignment
+    balances the CTAs to within one pair and is as fast or faster; in between
+    (e.g. one batch of 32 heads at N = 8192) the greedy claims balance
+    better."""
     if schedule not in ("auto", "static", "dynamic"):
         raise ValueError("schedule must be 'auto', 'static' or 'dynamic'")
     if schedule != "auto":
         return schedule
     units = B * H * ((N + UNIT_ROWS - 1) // UNIT_ROWS)
-    return "dynamic" if units >= AUTO_DYNAMIC_UNITS_PER_SM * sm_count else "static"
+    lo, hi = AUTO_DYNAMIC_UNITS_PER_SM
+    return "dynamic" if lo * sm_count <= units < hi * sm_count else "static"
 
 
 def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,

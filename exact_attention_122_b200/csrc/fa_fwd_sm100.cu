@@ -81,29 +81,6 @@ constexpr int SW_COLS = 64;        // bf16 elements per 128-byte swizzled row
 // stays below 2^RESCALE_LOG2 and O is rescaled rarely.  l and O share the
 // stale reference, so O = acc / l and LSE = (m + log2 l) ln 2 stay exact.
 constexpr float RESCALE_LOG2 = 8.0f;
-// Columns of every 32-column chunk of an unmasked score row whose
-// exponential is computed by exp2_poly instead of MUFU ex2.
-// Measured on B200: every nonzero setting was slower on the long causal
-// workloads (the softmax is not MUFU-bound once the rescale is lazy), so the
-// default is 0; the polynomial path stays for tuning other shapes.
-#ifndef FA_POLY_COLS
-#define FA_POLY_COLS 0
-#endif
-#ifndef FA_MAX3
-#define FA_MAX3 0
-#endif
-constexpr int POLY_COLS = FA_POLY_COLS;
-static_assert(POLY_COLS >= 0 && POLY_COLS <= 32 && POLY_COLS % 2 == 0, "poly columns");
-
-// P is handed to the MMA thread in P_CHUNKS pieces of BN / P_CHUNKS keys, each
-// with its own barrier, so the P V products of a tile's first keys run on the
-// tensor core while the exponentials of its last keys are still being taken.
-#ifndef FA_PCHUNK
-#define FA_PCHUNK 1
-#endif
-constexpr int P_CHUNKS = FA_PCHUNK ? 4 : 1;
-constexpr int P_CHUNK_KEYS = BN / P_CHUNKS;
-
 enum : uint32_t {
     ROLE_SOFTMAX = 1u, ROLE_MMA = 2u, ROLE_PRODUCER = 3u, ROLE_DRAIN = 4u
 };
@@ -132,8 +109,8 @@ struct Layout {
     static constexpr int B_Q_FULL = 2 * NS;
     static constexpr int B_Q_EMPTY = 2 * NS + 1;
     static constexpr int B_S_FULL = 2 * NS + 2;      // [2]
-    static constexpr int B_P_FULL = 2 * NS + 4;      // [2][P_CHUNKS]
-    static constexpr int B_O_FULL = B_P_FULL + 2 * P_CHUNKS;   // [2]
+    static constexpr int B_P_FULL = 2 * NS + 4;      // [2]
+    static constexpr int B_O_FULL = B_P_FULL + 2;    // [2]
     static constexpr int B_O_EMPTY = B_O_FULL + 2;   // [2]
     static constexpr int B_DRAIN = B_O_EMPTY + 2;
     static constexpr int B_UFULL = B_DRAIN + 1;      // [2] unit queue (dynamic schedule)
@@ -181,40 +158,6 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Watchd
 // Barrier 0 over all NUM_THREADS threads, usable from different branches.
 __device__ __forceinline__ void cta_sync() {
     asm volatile("bar.sync 0, %0;" ::"n"(NUM_THREADS) : "memory");
-}
-
-// Software 2^x on the FMA pipe for a packed pair, used for part of each
-// score row so the MUFU unit (ex2) is not the only source of exponentials.
-// Method: Cody-Waite range reduction x = n + f with n = rint(x) (the
-// 1.5 * 2^23 shifter), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
-// coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
-// exchange; csrc/gen_exp2_poly.py reproduces them, max relative error
-// 7.5e-5, below the 2^-9 rounding of the bf16 P it feeds); 2^n is added to
-// the exponent field with one integer multiply-add per value (the shifter's
-// own bits vanish: they sit above bit 8 of t).  The floating-point steps run
-// as f32x2 pairs.  Valid for x in [-126, 64]; inputs below -126 are clamped
-// (results below 2^-125 are meaningless there, so the kernel only uses it on
-// tiles without masked scores).
-constexpr float EXP2_C0 = 9.999280572e-01f;
-constexpr float EXP2_C1 = 6.932609677e-01f;
-constexpr float EXP2_C2 = 2.426111251e-01f;
-constexpr float EXP2_C3 = 5.517166853e-02f;
-
-__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& y0, float& y1) {
-    float x0, x1;
-    f2_unpack(x2, x0, x1);
-    const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-    const uint64_t sh = f2_pack(12582912.0f, 12582912.0f);         // 1.5 * 2^23
-    const uint64_t t = f2_add(xc, sh);           // low mantissa bits of t hold rint(x)
-    const uint64_t f = f2_sub(xc, f2_sub(t, sh));
-    uint64_t p = f2_fma(f2_pack(EXP2_C3, EXP2_C3), f, f2_pack(EXP2_C2, EXP2_C2));
-    p = f2_fma(p, f, f2_pack(EXP2_C1, EXP2_C1));
-    p = f2_fma(p, f, f2_pack(EXP2_C0, EXP2_C0));
-    float p0, p1, t0, t1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(t, t0, t1);
-    y0 = __uint_as_float(__float_as_uint(p0) + __float_as_uint(t0) * (1u << 23));
-    y1 = __uint_as_float(__float_as_uint(p1) + __float_as_uint(t1) * (1u << 23));
 }
 
 // ---------------------------------------------------------------------------
@@ -315,28 +258,22 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint6
     }
 }
 
-// O += P V for one sub-tile over keys [c * P_CHUNK_KEYS, (c + 1) *
-// P_CHUNK_KEYS) of the tile: A = P from TMEM (8 columns per step: 16 keys as
-// bf16 pairs, or 32 keys as FP8 quads).  bf16: B = V MN-major, 16 key rows of
-// 128 bytes per step.  FP8: B = V^T K-major (d rows of 128 keys), a step is
-// 32 bytes inside the swizzled rows.  `first`: the tile's first chunk of a
-// unit's first tile overwrites O instead of accumulating.
+// O += P V for one sub-tile: A = P from TMEM (8 columns per step: 16 keys
+// as bf16 pairs, or 32 keys as FP8 quads).  bf16: B = V MN-major, 16 key
+// rows of 128 bytes per step.  FP8: B = V^T K-major (d rows of 128 keys), a
+// step is 32 bytes inside the swizzled rows.  `first`: the unit's first tile
+// overwrites O instead of accumulating.
 template <bool F8>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc,
-                                         uint32_t idesc, int c, bool first) {
+                                         uint32_t idesc, bool first) {
     if constexpr (F8) {
-        constexpr int STEPS = P_CHUNK_KEYS / 32;
 #pragma unroll
-        for (int i = 0; i < STEPS; ++i) {
-            const int kk = c * STEPS + i;
+        for (int kk = 0; kk < BN / 32; ++kk)
             mma_ts_f8(o_tmem, p_tmem + kk * 8, desc_add(v_desc, uint32_t((kk * 32) >> 4)), idesc,
                       (first && kk == 0) ? 0u : 1u);
-        }
     } else {
-        constexpr int STEPS = P_CHUNK_KEYS / 16;
 #pragma unroll
-        for (int i = 0; i < STEPS; ++i) {
-            const int kk = c * STEPS + i;
+        for (int kk = 0; kk < BN / 16; ++kk) {
             const uint32_t off = uint32_t((kk * 16 * 128) >> 4);
             mma_ts(o_tmem, p_tmem + kk * 8, desc_add(v_desc, off), idesc,
                    (first && kk == 0) ? 0u : 1u);
@@ -362,14 +299,11 @@ __device__ __forceinline__ float round_as_p(float p) {
 // P = 2^(s * scale_log2 - m) for one score row held in registers, written
 // to TMEM over the row's first columns: bf16 pairs (64 columns) or, with F8,
 // FP8 E4M3 quads (32 columns).  The row sum (of the unrounded fp32 P) goes to
-// four packed partial accumulators.  The first NPOLY columns of every
-// 32-column chunk use exp2_poly_x2, the rest MUFU ex2.  Each chunk of
-// P_CHUNK_KEYS keys is published on its barrier (p_bar + 8 c) once its TMEM
-// stores have completed.
-template <int NPOLY, bool F8 = false>
+// four packed partial accumulators.  The caller waits for the TMEM stores
+// and publishes P.
+template <bool F8>
 __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_log2, float neg_m,
-                                             uint64_t (&acc)[4], uint32_t tS, uint32_t p_bar) {
-    static_assert(P_CHUNK_KEYS % 32 == 0, "P chunks are whole 32-key groups");
+                                             uint64_t (&acc)[4], uint32_t tS) {
     const uint64_t c2 = f2_pack(scale_log2, scale_log2);
     const uint64_t m2 = f2_pack(neg_m, neg_m);
     uint64_t pf_prev = 0;                        // F8: the previous pair of P values
@@ -380,13 +314,8 @@ __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_l
         for (int i = 0; i < 16; ++i) {
             float x0, x1;
             f2_unpack(f2_fma(f2_pack(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), c2, m2), x0, x1);
-            float p0, p1;
-            if (2 * i < NPOLY) {
-                exp2_poly_x2(f2_pack(x0, x1), p0, p1);
-            } else {
-                p0 = ex2(x0);
-                p1 = ex2(x1);
-            }
+            const float p0 = ex2(x0);
+            const float p1 = ex2(x1);
             acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
             if constexpr (F8) {
                 // keys 2i-2 .. 2i+1 go into word i/2 once both pairs exist
@@ -405,11 +334,136 @@ __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_l
             tmem_st8(tS + c * 8, pk);            // P (FP8) over S columns [0, 32)
         else
             tmem_st16(tS + c * 16, pk);          // P (bf16) over S columns [0, 64)
-        if ((c + 1) % (P_CHUNK_KEYS / 32) == 0) {
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(p_bar + 8u * uint32_t(c / (P_CHUNK_KEYS / 32)));
+    }
+}
+
+// One K/V tile of the online softmax for the row held in s[] (the thread's
+// TMEM lane): mask (keys past N_k on the last tile; causal keys past the row's
+// limit on tiles that cross the sub-tile's first limit), row max, lazy rescale
+// of the reference m and of O in TMEM, P into TMEM over S, publication of P on
+// p_bar, then the row sums.  a: the sub-tile's first row; row: this thread's
+// row.
+template <int D, bool F8>
+__device__ __forceinline__ void softmax_tile(float (&s)[BN], int j, int nkb, int Nk, int causal,
+                                             int a, int row, int koff, float scale_log2, float& m,
+                                             float& l, float& lc, uint32_t tS, uint32_t tO,
+                                             uint32_t p_bar) {
+    // Mask: keys beyond N_k on the last tile; causal: keys past
+    // the row's limit on the tiles that cross the sub-tile's
+    // first limit (the diagonal).
+    const bool tail = (j == nkb - 1) && (Nk % BN != 0);
+    const bool diag = causal && (j * BN + BN - 1 > a + koff);
+    if (tail || diag) {
+        const int lim_tail = Nk - j * BN;          // key c allowed iff c < lim_tail
+        const int lim_diag = row + koff - j * BN;  // key c allowed iff c <= lim_diag
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+            const bool bad = (c >= lim_tail) || (causal && c > lim_diag);
+            s[c] = bad ? -INFINITY : s[c];
         }
+    }
+    // Row max: eight chains of three-input max (chain i takes
+    // columns i, i+8, ..., i+120; one instruction folds two
+    // columns), then a tree.
+    float mx8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx8[i] = fmax3(s[i], s[8 + i], s[16 + i]);
+#pragma unroll
+    for (int c = 24; c < BN - 8; c += 16) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[c + i], s[c + 8 + i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], s[BN - 8 + i]);
+    const float s_top = fmaxf(fmax3(fmax3(mx8[0], mx8[1], mx8[2]),
+                                    fmax3(mx8[3], mx8[4], mx8[5]), mx8[6]),
+                              mx8[7]);
+    const float m_blk = s_top * scale_log2;
+    // Lazy rescale: the reference m (that l and O refer to) moves
+    // to the row's new maximum only when some row of the warp
+    // exceeds it by more than RESCALE_LOG2 (first tile: m = -inf,
+    // so every lane moves).  O is then rescaled in TMEM: the P V
+    // of tile j-1 is complete, its commit preceded the S_t commit
+    // waited on above.
+    if (__any_sync(0xffffffffu, m_blk > m + RESCALE_LOG2)) {
+        const float m_new = fmaxf(m, m_blk);
+        const float alpha = ex2(m - m_new);      // 0 on the first tile
+        if (j > 0) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tO + c * 32, r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                tmem_st32(tO + c * 32, r);
+            }
+        }
+        l *= alpha;
+        lc *= alpha;
+        m = m_new;
+    }
+    uint64_t acc[4] = {0, 0, 0, 0};              // four packed (0.f, 0.f)
+    exp_row_to_p<F8>(s, scale_log2, -m, acc, tS);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(p_bar);
+    // The P V product takes P rounded to its operand type, while
+    // l sums the unrounded P.  O is normalised by l + lc, lc
+    // holding the rounding error of each tile's largest P: with a
+    // stale reference m that P is not a power of two, and when it
+    // dominates the row (peaked attention) its rounding then
+    // cancels between O's numerator and normaliser.  The LSE
+    // keeps the unrounded l.
+    {
+        const float p_top = ex2(fmaf(s_top, scale_log2, -m));
+        lc += round_as_p<F8>(p_top) - p_top;
+    }
+    {
+        float a0, a1, a2, a3, a4, a5, a6, a7;
+        f2_unpack(acc[0], a0, a1);
+        f2_unpack(acc[1], a2, a3);
+        f2_unpack(acc[2], a4, a5);
+        f2_unpack(acc[3], a6, a7);
+        l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+    }
+}
+
+// Epilogue of one row: O / (l + lc) -> bf16 -> the row of o_head (element
+// stride o_sn between rows), LSE = (m + log2 l) ln 2 -> lse_head[row]; rows
+// at or past N_q are not stored.  o_scale multiplies O (FP8: V's scale).
+template <int D, bool F8>
+__device__ __forceinline__ void store_o_row(uint32_t tO, __nv_bfloat16* o_head, float* lse_head,
+                                            int row, int Nq, long long o_sn, float m, float l,
+                                            float lc, float o_scale) {
+    float inv_l = 1.f / (l + lc);
+    if constexpr (F8) inv_l *= o_scale;
+    const bool store = row < Nq;
+    __nv_bfloat16* orow = o_head + (long long)(store ? row : 0) * o_sn;
+    uint32_t ro[D];
+    if constexpr (D == 128) {
+        tmem_ld128(tO, ro);
+    } else {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ro[c * 32 + i] = r[i];
+        }
+    }
+    if (store) {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+        for (int v4 = 0; v4 < D / 8; ++v4) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(ro[8 * v4 + 2 * i]) * inv_l,
+                                    __uint_as_float(ro[8 * v4 + 2 * i + 1]) * inv_l);
+            dst[v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        lse_head[row] = (m + log2f(l)) * 0.69314718055994530942f;
     }
 }
 
@@ -487,7 +541,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_init(bar(L::B_Q_EMPTY), 1);
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(L::B_S_FULL + t), 1);
-            for (int c = 0; c < P_CHUNKS; ++c) mbar_init(bar(L::B_P_FULL + t * P_CHUNKS + c), BM);
+            mbar_init(bar(L::B_P_FULL + t), BM);
             mbar_init(bar(L::B_O_FULL + t), 1);
             mbar_init(bar(L::B_O_EMPTY + t), BM);
         }
@@ -626,17 +680,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t stage_step = uint32_t(L::KV_BYTES >> 4);
             const uint32_t tS0 = tmem + L::TM_S0, tS1 = tmem + L::TM_S1;
             const uint32_t tO0 = tmem + L::TM_O0, tO1 = tmem + L::TM_O1;
-            // O_t += P_t V for one tile, each chunk of keys as soon as the
-            // softmax warpgroup has published its part of P_t.
-            auto pv_chunks = [&](int t, uint32_t pcnt, uint32_t tO, uint32_t tS, uint64_t v_desc,
-                                 bool first, int u) -> bool {
-#pragma unroll
-                for (int c = 0; c < P_CHUNKS; ++c) {
-                    if (!wait_phase(bar(L::B_P_FULL + t * P_CHUNKS + c), pcnt & 1u, wd, ROLE_MMA, u))
-                        return false;
-                    tc_fence_after();
-                    issue_pv<F8>(tO, tS, v_desc, ID_PV, c, first);
-                }
+            // O_t += P_t V for one tile once the softmax warpgroup has
+            // published P_t.
+            auto pv = [&](int t, uint32_t pcnt, uint32_t tO, uint32_t tS, uint64_t v_desc,
+                          bool first, int u) -> bool {
+                if (!wait_phase(bar(L::B_P_FULL + t), pcnt & 1u, wd, ROLE_MMA, u)) return false;
+                tc_fence_after();
+                issue_pv<F8>(tO, tS, v_desc, ID_PV, first);
                 return true;
             };
             for (int kq = 0; ok; ++kq, ++units) {
@@ -665,26 +715,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     ++cons;
                     const bool next = j + 1 < w.nb1;
-                    if (next) {
+                    // K_{j+1} is waited for only when the first S of tile
+                    // j+1 is issued, after P V of tile j.
+                    bool have_k = false;
+                    auto wait_next_k = [&]() -> bool {
+                        if (have_k) return true;
                         sK = cons % NS;
-                        if (!wait_phase(bar(L::B_KV_FULL + sK), (cons / NS) & 1u, wd, ROLE_MMA, u)) {
-                            ok = false;
-                            break;
-                        }
+                        if (!wait_phase(bar(L::B_KV_FULL + sK), (cons / NS) & 1u, wd, ROLE_MMA, u))
+                            return false;
                         ++cons;
-                    }
+                        have_k = true;
+                        return true;
+                    };
                     if (j < w.nb0) {
                         if (j == 0 && !wait_phase(bar(L::B_O_EMPTY + 0), (units & 1u) ^ 1u, wd,
                                                   ROLE_MMA, u)) {
                             ok = false;
                             break;
                         }
-                        if (!pv_chunks(0, pcnt0, tO0, tS0, desc_add(dv0, sV * stage_step), j == 0, u)) {
+                        if (!pv(0, pcnt0, tO0, tS0, desc_add(dv0, sV * stage_step), j == 0, u)) {
                             ok = false;
                             break;
                         }
                         ++pcnt0;
                         if (j + 1 < w.nb0) {
+                            if (!wait_next_k()) {
+                                ok = false;
+                                break;
+                            }
                             issue_qk<L::QK_STEPS, L::HALF_BYTES, F8>(tS0, dq0, desc_add(dk0, sK * stage_step), ID_S);
                             tc_commit(bar(L::B_S_FULL + 0));
                         }
@@ -694,16 +752,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                         break;
                     }
-                    if (!pv_chunks(1, pcnt1, tO1, tS1, desc_add(dv0, sV * stage_step), j == 0, u)) {
+                    if (!pv(1, pcnt1, tO1, tS1, desc_add(dv0, sV * stage_step), j == 0, u)) {
                         ok = false;
                         break;
                     }
                     ++pcnt1;
+                    // V_j is free once both P V products have read it: its
+                    // stage is released before S_1(j+1) is queued, so the
+                    // producer refills it one QK^T group earlier.
+                    tc_commit(bar(L::B_KV_EMPTY + sV));
                     if (next) {
+                        if (!wait_next_k()) {
+                            ok = false;
+                            break;
+                        }
                         issue_qk<L::QK_STEPS, L::HALF_BYTES, F8>(tS1, dq1, desc_add(dk0, sK * stage_step), ID_S);
                         tc_commit(bar(L::B_S_FULL + 1));
                     }
-                    tc_commit(bar(L::B_KV_EMPTY + sV));
                     if (next) tc_commit(bar(L::B_KV_EMPTY + sK));
                     if (next && j + 1 == w.nb1 - 1) tc_commit(bar(L::B_Q_EMPTY));
                     if (j == w.nb1 - 1) tc_commit(bar(L::B_O_FULL + 1));
@@ -762,96 +827,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
                 }
-                // Mask: keys beyond N_k on the last tile; causal: keys past
-                // the row's limit on the tiles that cross the sub-tile's
-                // first limit (the diagonal).
-                const bool tail = (j == nkb - 1) && (Nk % BN != 0);
-                const bool diag = causal && (j * BN + BN - 1 > a + koff);
-                if (tail || diag) {
-                    const int lim_tail = Nk - j * BN;          // key c allowed iff c < lim_tail
-                    const int lim_diag = row + koff - j * BN;  // key c allowed iff c <= lim_diag
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) {
-                        const bool bad = (c >= lim_tail) || (causal && c > lim_diag);
-                        s[c] = bad ? -INFINITY : s[c];
-                    }
-                }
-                // Row max: eight independent chains, then a tree.
-                float mx8[8];
-#if FA_MAX3
-                // three-input max: about half the instructions of two-input
-                // chains.  Chain i takes columns i, i+8, ..., i+120.
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx8[i] = fmax3(s[i], s[8 + i], s[16 + i]);
-#pragma unroll
-                for (int c = 24; c < BN - 8; c += 16) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[c + i], s[c + 8 + i]);
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], s[BN - 8 + i]);
-                const float s_top = fmaxf(fmax3(fmax3(mx8[0], mx8[1], mx8[2]),
-                                                fmax3(mx8[3], mx8[4], mx8[5]), mx8[6]),
-                                          mx8[7]);
-#else
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx8[i] = s[i];
-#pragma unroll
-                for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-                const float s_top =
-                    fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-#endif
-                const float m_blk = s_top * scale_log2;
-                // Lazy rescale (first tile: m = -inf, so every lane moves).
-                if (__any_sync(0xffffffffu, m_blk > m + RESCALE_LOG2)) {
-                    const float m_new = fmaxf(m, m_blk);
-                    const float alpha = ex2(m - m_new);      // 0 on the first tile
-                    if (j > 0) {
-                        // The PV of tile j-1 is complete: its commit
-                        // preceded the S_t commit waited on above.
-#pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t r[32];
-                            tmem_ld32(tO + c * 32, r);
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                            tmem_st32(tO + c * 32, r);
-                        }
-                    }
-                    l *= alpha;
-                    lc *= alpha;
-                    m = m_new;
-                }
-                const float neg_m = -m;
-                // The P V product takes P rounded to its operand type, while
-                // l sums the unrounded P.  O is normalised by l + lc, lc
-                // holding the rounding error of each tile's largest P: with a
-                // stale reference m that P is not a power of two, and when it
-                // dominates the row (peaked attention) its rounding then
-                // cancels between O's numerator and normaliser.  The LSE
-                // keeps the unrounded l.
-                {
-                    const float p_top = ex2(fmaf(s_top, scale_log2, neg_m));
-                    lc += round_as_p<F8>(p_top) - p_top;
-                }
-                uint64_t acc[4] = {0, 0, 0, 0};              // four packed (0.f, 0.f)
-                // Tiles without masked scores may use the FMA-pipe 2^x for
-                // part of the row; the choice is warp-uniform, made once.
-                const uint32_t p_bar = bar(L::B_P_FULL + t * P_CHUNKS);
-                if (POLY_COLS > 0 && !(tail || diag))
-                    exp_row_to_p<POLY_COLS, F8>(s, scale_log2, neg_m, acc, tS, p_bar);
-                else
-                    exp_row_to_p<0, F8>(s, scale_log2, neg_m, acc, tS, p_bar);
-                {
-                    float a0, a1, a2, a3, a4, a5, a6, a7;
-                    f2_unpack(acc[0], a0, a1);
-                    f2_unpack(acc[1], a2, a3);
-                    f2_unpack(acc[2], a4, a5);
-                    f2_unpack(acc[3], a6, a7);
-                    l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
-                }
+                softmax_tile<D, F8>(s, j, nkb, Nk, causal, a, row, koff, scale_log2, m, l, lc, tS,
+                                    tO, bar(L::B_P_FULL + t));
             }
             if (!ok) break;
             // Epilogue: O / l -> bf16 -> global; LSE.
@@ -859,36 +836,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ++ocnt;
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
             tc_fence_after();
-            float inv_l = 1.f / (l + lc);
-            if constexpr (F8) inv_l *= o_scale;
-            const bool store = row < Nq;
             const int wb = w.bh / H, wh = w.bh - (w.bh / H) * H;     // batch, head
-            __nv_bfloat16* orow = Og + wb * o_sb + wh * o_sh + (long long)(store ? row : 0) * o_sn;
-            uint32_t ro[D];
-            if constexpr (D == 128) {
-                tmem_ld128(tO, ro);
-            } else {
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tO + c * 32, r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ro[c * 32 + i] = r[i];
-                }
-            }
-            if (store) {
-                uint4* dst = reinterpret_cast<uint4*>(orow);
-#pragma unroll
-                for (int v4 = 0; v4 < D / 8; ++v4) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        pk[i] = pack_bf16x2(__uint_as_float(ro[8 * v4 + 2 * i]) * inv_l,
-                                            __uint_as_float(ro[8 * v4 + 2 * i + 1]) * inv_l);
-                    dst[v4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-            }
-            if (store) LSEg[size_t(w.bh) * Nq + row] = (m + log2f(l)) * 0.69314718055994530942f;
+            store_o_row<D, F8>(tO, Og + wb * o_sb + wh * o_sh, LSEg + size_t(w.bh) * Nq, row, Nq,
+                               o_sn, m, l, lc, o_scale);
             tc_fence_before();
             mbar_arrive(bar(L::B_O_EMPTY + t));
         }
@@ -1021,10 +971,10 @@ namespace {
 // per shape.
 struct HgKey {
     long long BH;
-    int Nq, Nk, D, causal, grid;
+    int Nq, Nk, D, causal, grid, unit_rows;
     bool operator==(const HgKey& o) const {
         return BH == o.BH && Nq == o.Nq && Nk == o.Nk && D == o.D && causal == o.causal &&
-               grid == o.grid;
+               grid == o.grid && unit_rows == o.unit_rows;
     }
 };
 struct StaticPlan {
@@ -1038,16 +988,18 @@ int g_hg_count = 0;
 
 // Max CTA load over mean CTA load of the static assignment, replayed.
 double static_imbalance(long long BH, int Nq, int Nk, int causal, long long hg, int paired,
-                        int grid) {
-    const long long nq2 = (Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+                        int grid, int unit_rows) {
+    const long long nq2 = (Nq + unit_rows - 1) / unit_rows;
     const long long nkb = (Nk + fa::BN - 1) / fa::BN;
     const long long off = Nk - Nq;
     std::vector<long long> load(size_t(grid), 0);
-    auto cost = [&](long long qb2) {            // K/V tiles of both sub-tiles + overhead
-        const long long r0 = qb2 * fa::UNIT_ROWS;
-        const long long nb0 = causal ? std::min((r0 + fa::BM - 1 + off) / fa::BN + 1, nkb) : nkb;
-        const long long nb1 =
-            causal ? std::min((r0 + 2 * fa::BM - 1 + off) / fa::BN + 1, nkb) : nkb;
+    // K/V tiles of both sub-tiles (the tiles of each half unit's last row)
+    // plus a fixed per-unit overhead.
+    auto cost = [&](long long qb2) {
+        const long long r0 = qb2 * unit_rows;
+        const long long half = unit_rows / 2;
+        const long long nb0 = causal ? std::min((r0 + half - 1 + off) / fa::BN + 1, nkb) : nkb;
+        const long long nb1 = causal ? std::min((r0 + unit_rows - 1 + off) / fa::BN + 1, nkb) : nkb;
         return nb0 + nb1 + 2;
     };
     if (!paired) {
@@ -1082,8 +1034,9 @@ double static_imbalance(long long BH, int Nq, int Nk, int causal, long long hg, 
     return double(mx) * grid / double(sum);
 }
 
-StaticPlan choose_static_plan(long long BH, int Nq, int Nk, int D, int causal, int grid) {
-    const HgKey key{BH, Nq, Nk, D, causal, grid};
+StaticPlan choose_static_plan(long long BH, int Nq, int Nk, int D, int causal, int grid,
+                              int unit_rows) {
+    const HgKey key{BH, Nq, Nk, D, causal, grid, unit_rows};
     {
         std::lock_guard<std::mutex> lk(g_hg_mutex);
         for (int i = 0; i < g_hg_count; ++i)
@@ -1094,7 +1047,7 @@ StaticPlan choose_static_plan(long long BH, int Nq, int Nk, int D, int causal, i
     double best_cost = 1e30;
     // Bound the replay work for very large problems: beyond ~4M units the
     // assignment statistics no longer depend on hg, so all heads form one group.
-    const long long units = ((Nq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS) * BH;
+    const long long units = ((Nq + unit_rows - 1) / unit_rows) * BH;
     if (units <= (4LL << 20)) {
         for (int paired = 0; paired <= (causal ? 1 : 0); ++paired) {
             for (long long hg = 1;; hg = std::min(hg * 2, BH)) {
@@ -1104,7 +1057,7 @@ StaticPlan choose_static_plan(long long BH, int Nq, int Nk, int D, int causal, i
                                  : ws <= 64.0 * (1 << 20) ? 0.06
                                  : ws <= 128.0 * (1 << 20) ? 0.09 : 0.12;
                 const double cost =
-                    static_imbalance(BH, Nq, Nk, causal, hg, paired, grid) * (1.0 + pen);
+                    static_imbalance(BH, Nq, Nk, causal, hg, paired, grid, unit_rows) * (1.0 + pen);
                 if (cost < best_cost - 1e-9) {
                     best_cost = cost;
                     best = StaticPlan{hg, paired};
@@ -1158,7 +1111,7 @@ fa_status launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     if (sched)
         plan.hg = (BH * kv_head_bytes <= (32LL << 20)) ? BH : (16LL << 20) / kv_head_bytes;
     else
-        plan = choose_static_plan(BH, Nq, Nk, D, causal, grid);
+        plan = choose_static_plan(BH, Nq, Nk, D, causal, grid, fa::UNIT_ROWS);
 #ifdef FA_HEAD_GROUP
     plan.hg = FA_HEAD_GROUP;
 #endif

@@ -142,19 +142,24 @@ def test_l2_rotation_plan():
 
 
 def test_auto_schedule_resolution():
-    """"auto" picks the dynamic schedule from 4 units of 256 rows per SM."""
+    """"auto" picks the dynamic schedule from 4 to 12 units of 256 rows per SM."""
     from exact_attention_122_b200 import resolve_schedule
 
-    assert resolve_schedule("auto", 2, 32, 8192, 148) == "dynamic"     # 2048 units
+    assert resolve_schedule("auto", 2, 32, 8192, 148) == "static"      # 2048 units >= 12 x 148
     assert resolve_schedule("auto", 1, 32, 8192, 148) == "dynamic"     # 1024
     assert resolve_schedule("auto", 1, 32, 4096, 148) == "static"      # 512 < 592
     assert resolve_schedule("auto", 8, 12, 1024, 148) == "static"      # 384
     assert resolve_schedule("auto", 1, 37, 4096, 148) == "dynamic"     # 592 = 4 x 148
     assert resolve_schedule("auto", 1, 37, 4095, 148) == "dynamic"     # ceil(4095/256) = 16
     assert resolve_schedule("auto", 1, 37, 3840, 148) == "static"      # 555
+    assert resolve_schedule("auto", 1, 16, 32768, 148) == "static"     # 2048
+    assert resolve_schedule("auto", 1, 111, 4096, 148) == "static"     # 1776 = 12 x 148
+    assert resolve_schedule("auto", 1, 111, 4095, 148) == "static"     # ceil(4095/256) = 16
+    assert resolve_schedule("auto", 1, 110, 4096, 148) == "dynamic"    # 1760 < 1776
     for s in ("static", "dynamic"):
         assert resolve_schedule(s, 1, 1, 1, 148) == s
     with pytest.raises(ValueError):
         resolve_schedule("fast", 1, 1, 1, 148)
-    assert bench.bench_schedule("auto", synth.workload(4)) == "dynamic"
+    assert bench.bench_schedule("auto", synth.workload(4)) == "static"
+    assert bench.bench_schedule("auto", synth.workload(5)) == "static"
     assert bench.bench_schedule("auto", synth.workload(2)) == "static"

@@ -43,7 +43,7 @@ print("all raised")
 def test_package_never_imports_the_oracle():
     """No module of the package imports the oracle; the runtime modules (the
     binding, autograd, build) do not even import numpy.  csrc/ holds only the
-    CUDA sources and the generator of the exp2 polynomial's coefficients."""
+    CUDA sources."""
     oracle_pat = re.compile(r"^\s*(import\s+oracle|from\s+oracle\b)", re.M)
     numpy_pat = re.compile(r"^\s*(import\s+numpy|from\s+numpy\b)", re.M)
     for dirpath, _, files in os.walk(PKG):
