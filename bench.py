@@ -573,6 +573,11 @@ def run_decode(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     w = synth.DECODE_WORKLOAD
+    if args.decode_batch != w.B:
+        # a smaller batch of the same shape (profiling captures); traffic
+        # and time scale with the batch
+        w = synth.DecodeWorkload(f"{w.name}_b{args.decode_batch}", args.decode_batch, w.H, w.Nq,
+                                 w.Nk, w.d, w.causal, w.seed)
     q, k, v = (t.to(dev) for t in synth.draw_decode_qkv(w.B, w.H, w.Nq, w.Nk, w.d, w.seed))
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
@@ -835,6 +840,9 @@ def main(argv=None):
                          "(graph-replayed): the L2-warm figure for workloads that fit in L2")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode-shaped path (HBM-bound) instead of the headline line")
+    ap.add_argument("--decode-batch", type=int, default=synth.DECODE_WORKLOAD.B,
+                    help="batch of the --decode line (default: the decode workload's); smaller "
+                         "batches keep profiling captures to a few GB")
     ap.add_argument("--fp8", action="store_true",
                     help="time the FP8 (E4M3) forward of the workload's shape")
     ap.add_argument("--bwd", action="store_true",
