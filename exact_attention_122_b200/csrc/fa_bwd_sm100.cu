@@ -512,9 +512,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                         mma_ss(tmem + C::TM_DQ, desc_add(ds_mn, off), desc_add(dK_mn, off), ID_Q,
                                kk > 0 ? 1u : 0u);
                 }
+                // One commit for the block's gradients: the dQ warps, which
+                // wait on it every step, pass the release of the dS buffer and
+                // of the Q / dO stage on with plain arrivals (each commit costs
+                // tensor-pipe time).
                 tc_commit(bar(C::B_DQ_FULL));
-                tc_commit(bar(C::B_DS_FREE + db));
-                tc_commit(bar(C::B_QD_EMPTY + s));
                 return true;
             };
 
@@ -569,6 +571,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int n = 0; n < nsteps; ++n) {
             if (!warp_wait(bar(C::B_DQ_FULL), n & 1, wd, ROLE_DQ, blk_id)) break;
             tc_fence_after();
+            if (qw == 0 && lane == 0) {
+                // block n's dV, dK and dQ products are complete: its dS
+                // buffer and its Q / dO stage are free
+                mbar_arrive(bar(C::B_DS_FREE + (n % 2)));
+                mbar_arrive(bar(C::B_QD_EMPTY + (n % NS)));
+            }
             const int q0 = (qb_first + n) * BQ;
             if (C::DQ_T) {
                 // lane = d index t; columns = the BQ queries of the block
