@@ -389,14 +389,16 @@ __device__ __forceinline__ void softmax_tile(float (&s)[BN], int j, int nkb, int
         const float m_new = fmaxf(m, m_blk);
         const float alpha = ex2(m - m_new);      // 0 on the first tile
         if (j > 0) {
+            // 16 columns at a time: with the score row live, wider chunks
+            // push the softmax warps past their register budget (spills).
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tO + c * 32, r);
+            for (int c = 0; c < D / 16; ++c) {
+                uint32_t r[16];
+                tmem_ld16(tO + c * 16, r);
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
+                for (int i = 0; i < 16; ++i)
                     r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                tmem_st32(tO + c * 32, r);
+                tmem_st16(tO + c * 16, r);
             }
         }
         l *= alpha;
