@@ -770,6 +770,509 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 }
 
 // ---------------------------------------------------------------------------
+// d = 128 kernel: 128 query rows per step, every MMA at M = N = 128.
+//
+// TMEM holds dQ, dV and dK (128 columns each) and one 128-column region X
+// that serves, in turn, S^T of the step, dP^T of the step (once the compute
+// warps have read S^T), and P as bf16 pairs (written by each compute warp
+// over the dP^T columns it has already read).  K stays in shared memory, so
+// S^T = K Q^T and dP^T = V dO^T are SS products.  Per step n the MMA thread
+// issues
+//   S^T(n) | dQ(n-1) | (S^T read) dP^T(n) | (P, dS written) dV(n), dK(n)
+// so the compute warps' exponentials of step n overlap the tensor core's dQ
+// of step n-1 and dP^T of step n; dV(n), issued before S^T(n+1) that
+// overwrites X, has read P(n) first (MMAs from one thread run in issue
+// order); and the Q / dO stage of step n is released right after dK(n), a
+// whole step before the next S^T needs the refill.
+// 512 threads: warps 0-7 compute, 8-11 dQ drain, 12 MMA, 13 TMA, 14-15 idle;
+// the compute warpgroups take 176 registers, the dQ warpgroup 64 and the
+// last warpgroup 88 (setmaxnreg, from 128 at launch).
+// ---------------------------------------------------------------------------
+struct CfgX {
+    static constexpr int D = 128;
+    static constexpr int BQ = 128;
+    static constexpr int NSX = 2;                        // Q / dO stages
+    static constexpr int THREADS = 512;
+    static constexpr int REGS_LAUNCH = 128;
+    static constexpr int REGS_COMPUTE = 176;
+    static constexpr int REGS_DQ = 64;
+    static constexpr int REGS_OTHER = 88;
+    static_assert(256 * REGS_COMPUTE + 128 * REGS_DQ + 128 * REGS_OTHER <=
+                      THREADS * REGS_LAUNCH,
+                  "setmaxnreg split within the launch's registers");
+    static constexpr int KV_BYTES = BK * D * 2;          // 32 KiB
+    static constexpr int KV_SLAB = BK * 128;             // 64 columns of a K / V tile
+    static constexpr int QD_BYTES = BQ * D * 2;          // 32 KiB
+    static constexpr int QD_SLAB = BQ * 128;             // 64 columns of a Q / dO tile
+    static constexpr int DS_BYTES = BK * BQ * 2;         // 32 KiB
+    static constexpr int DS_SLAB = BK * 128;             // 64 queries of dS, all keys
+    static constexpr int VEC_BYTES = 2 * BQ * 4;         // -LSE2 and -D of one query block
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + KV_BYTES;
+    static constexpr int OFF_Q = OFF_V + KV_BYTES;
+    static constexpr int OFF_DO = OFF_Q + NSX * QD_BYTES;
+    static constexpr int OFF_DS = OFF_DO + NSX * QD_BYTES;
+    static constexpr int OFF_VEC = OFF_DS + DS_BYTES;
+    static constexpr int OFF_BAR = OFF_VEC + NSX * VEC_BYTES;
+    static constexpr int B_KV_FULL = 0;
+    static constexpr int B_QD_FULL = 1;                  // [NSX]
+    static constexpr int B_QD_EMPTY = 1 + NSX;           // [NSX]
+    static constexpr int B_S_FULL = 1 + 2 * NSX;
+    static constexpr int B_S_FREE = 2 + 2 * NSX;
+    static constexpr int B_DP_FULL = 3 + 2 * NSX;
+    static constexpr int B_DS_READY = 4 + 2 * NSX;
+    static constexpr int B_DQ_FULL = 5 + 2 * NSX;
+    static constexpr int B_DQ_EMPTY = 6 + 2 * NSX;
+    static constexpr int B_ACC_FULL = 7 + 2 * NSX;
+    static constexpr int B_DRAIN = 8 + 2 * NSX;
+    static constexpr int NUM_BARS = 9 + 2 * NSX;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem base, abort flag
+    static constexpr int BYTES = OFF_MISC + 16;
+    // The whole 227 KiB: what is left over after BYTES absorbs the rounding
+    // of the dynamic shared-memory base up to 1 KiB (checked in the kernel).
+    static constexpr int ALLOC = 227 * 1024;
+    static_assert(BYTES <= ALLOC, "shared memory budget");
+    static constexpr uint32_t TM_X = 0;                  // S^T, then dP^T, then P
+    static constexpr uint32_t TM_DQ = 128;               // dQ^T: d on the lanes
+    static constexpr uint32_t TM_DV = 256;
+    static constexpr uint32_t TM_DK = 384;
+    static constexpr uint32_t TM_COLS = 512;
+};
+
+// p = 2^(s * scale log2(e) - LSE2) for 32 query columns of one key row, with
+// the same masking as p_ds_chunk; kept in fp32 for dS.
+template <bool MASK>
+__device__ __forceinline__ void p_chunk(const uint32_t* sv, const float* nl, float cs, int qi0,
+                                        int key, int N, int causal, float* p) {
+    const uint64_t cs2 = f2_pack(cs, cs);
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(nl + j);
+        const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])),
+                                    cs2, f2_pack(l4.x, l4.y));
+        const uint64_t x23 = f2_fma(
+            f2_pack(__uint_as_float(sv[j + 2]), __uint_as_float(sv[j + 3])), cs2,
+            f2_pack(l4.z, l4.w));
+        float x[4];
+        f2_unpack(x01, x[0], x[1]);
+        f2_unpack(x23, x[2], x[3]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            p[j + u] = ex2(x[u]);
+            if (MASK) {
+                const int qi = qi0 + j + u;
+                if ((causal && qi < key) || qi >= N || key >= N) p[j + u] = 0.f;
+            }
+        }
+    }
+}
+
+// ds = p * (dP - D) for 32 query columns; P and dS rounded to bf16 pairs.
+__device__ __forceinline__ void ds_chunk(const float* p, const uint32_t* dpv,
+                                         const float* nd, uint32_t (&pu)[16],
+                                         uint32_t (&du)[16]) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+        const float4 d4 = *reinterpret_cast<const float4*>(nd + j);
+        const uint64_t t01 = f2_add(
+            f2_pack(__uint_as_float(dpv[j]), __uint_as_float(dpv[j + 1])), f2_pack(d4.x, d4.y));
+        const uint64_t t23 = f2_add(
+            f2_pack(__uint_as_float(dpv[j + 2]), __uint_as_float(dpv[j + 3])),
+            f2_pack(d4.z, d4.w));
+        float ds[4];
+        f2_unpack(f2_mul(f2_pack(p[j], p[j + 1]), t01), ds[0], ds[1]);
+        f2_unpack(f2_mul(f2_pack(p[j + 2], p[j + 3]), t23), ds[2], ds[3]);
+        pu[j / 2] = pack_bf16x2(p[j], p[j + 1]);
+        pu[j / 2 + 1] = pack_bf16x2(p[j + 2], p[j + 3]);
+        du[j / 2] = pack_bf16x2(ds[0], ds[1]);
+        du[j / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+    }
+}
+
+__device__ __forceinline__ void cta_sync_x() {
+    asm volatile("bar.sync 0, %0;" ::"n"(CfgX::THREADS) : "memory");
+}
+
+__global__ void __launch_bounds__(CfgX::THREADS, 1)
+bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+             const float* __restrict__ nlse2, const float* __restrict__ ndvec,
+             float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
+             __nv_bfloat16* __restrict__ dv, int BH, int H, int N, int Npad, int causal,
+             float scale, int hg, unsigned long long watchdog_ns, int inject, St3 sdk, St3 sdv) {
+    using X = CfgX;
+    constexpr int D = X::D;
+    constexpr int BQ = X::BQ;
+    constexpr int NSX = X::NSX;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // The layout needs BYTES from a 1 KiB boundary; the allocation leaves
+    // ALLOC - BYTES for the rounding.  If the base is placed worse than that,
+    // every thread leaves before touching shared memory or TMEM.
+    if (smem + X::BYTES > smem_raw + X::ALLOC) {
+        if (threadIdx.x == 0)
+            atomicCAS(&g_bwd_status, 0u, (uint32_t(FA_ERR_LAUNCH) << 24) | (ROLE_DRAIN << 20));
+        return;
+    }
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t bar0 = sbase + X::OFF_BAR;
+    auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + X::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + X::OFF_MISC + 4);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+
+    // Work order as in bwd_kernel: head groups of hg, key-block-major inside.
+    const int nkb = (N + BK - 1) / BK;
+    const int per_group = hg * nkb;
+    const int g = int(blockIdx.x) / per_group;
+    const int r_in = int(blockIdx.x) - g * per_group;
+    const int gh = min(hg, BH - g * hg);
+    const int kb = r_in / gh;
+    const int bh = g * hg + (r_in - kb * gh);
+    const int b = bh / H, h = bh - (bh / H) * H;
+    const int k0 = kb * BK;
+    const int nqb = (N + BQ - 1) / BQ;
+    const int qb_first = causal ? k0 / BQ : 0;
+    const int nsteps = nqb - qb_first;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(X::B_KV_FULL), 1);
+        for (int s = 0; s < NSX; ++s) {
+            mbar_init(bar(X::B_QD_FULL + s), 1);
+            mbar_init(bar(X::B_QD_EMPTY + s), 1);
+        }
+        mbar_init(bar(X::B_S_FULL), 1);
+        mbar_init(bar(X::B_S_FREE), COMPUTE_WARPS);
+        mbar_init(bar(X::B_DP_FULL), 1);
+        mbar_init(bar(X::B_DS_READY), COMPUTE_WARPS);
+        mbar_init(bar(X::B_DQ_FULL), 1);
+        mbar_init(bar(X::B_DQ_EMPTY), 4);
+        mbar_init(bar(X::B_ACC_FULL), 1);
+        mbar_init(bar(X::B_DRAIN), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(smem_addr(tmem_slot), X::TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    cta_sync_x();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Watchdog wd{abort_flag, watchdog_ns};
+    const uint32_t blk_id = blockIdx.x;
+
+    if (warp >= MMA_WARP) {
+        regs_dec<X::REGS_OTHER>();
+        if (warp == TMA_WARP && lane == 0) {
+            // ------------------------------------------------------------------
+            // Producer: K, V once; then Q, dO, -LSE2, -D of each query block.
+            // ------------------------------------------------------------------
+            mbar_arrive_expect_tx(bar(X::B_KV_FULL), 2 * X::KV_BYTES);
+#pragma unroll
+            for (int sl = 0; sl < D / 64; ++sl) {
+                tma_load_4d(sbase + X::OFF_K + sl * X::KV_SLAB, &tmK, sl * 64, k0, h, b,
+                            bar(X::B_KV_FULL));
+                tma_load_4d(sbase + X::OFF_V + sl * X::KV_SLAB, &tmV, sl * 64, k0, h, b,
+                            bar(X::B_KV_FULL));
+            }
+            int issued = 0;
+            // Host-chosen fault injection (inject = 1): CTA 0 never issues its
+            // first Q / dO block, so the waits on it can only end by the watchdog.
+            const bool skip0 = inject == 1 && blockIdx.x == 0;
+            for (int n = 0; n < nsteps; ++n) {
+                const int s = n % NSX;
+                if (n >= NSX && !wait_phase(bar(X::B_QD_EMPTY + s), ((n / NSX) - 1) & 1, wd,
+                                            ROLE_PRODUCER, blk_id))
+                    break;
+                ++issued;
+                if (skip0 && n == 0) continue;
+                const int q0 = (qb_first + n) * BQ;
+                const uint32_t full = bar(X::B_QD_FULL + s);
+                mbar_arrive_expect_tx(full, 2 * X::QD_BYTES + X::VEC_BYTES);
+#pragma unroll
+                for (int sl = 0; sl < D / 64; ++sl) {
+                    tma_load_4d(sbase + X::OFF_Q + s * X::QD_BYTES + sl * X::QD_SLAB, &tmQ,
+                                sl * 64, q0, h, b, full);
+                    tma_load_4d(sbase + X::OFF_DO + s * X::QD_BYTES + sl * X::QD_SLAB, &tmDO,
+                                sl * 64, q0, h, b, full);
+                }
+                const long long vrow = (long long)bh * Npad + q0;
+                bulk_load(sbase + X::OFF_VEC + s * X::VEC_BYTES, nlse2 + vrow, BQ * 4, full);
+                bulk_load(sbase + X::OFF_VEC + s * X::VEC_BYTES + BQ * 4, ndvec + vrow, BQ * 4,
+                          full);
+            }
+            // Drain: every copy this thread issued has landed before exit.
+            wait_drain(bar(X::B_KV_FULL), 0, watchdog_ns);
+            for (int n = (issued > NSX ? issued - NSX : 0); n < issued; ++n)
+                if (!(skip0 && n == 0))
+                    wait_drain(bar(X::B_QD_FULL + n % NSX), (n / NSX) & 1, watchdog_ns);
+        } else if (warp == MMA_WARP && lane == 0) {
+            // ------------------------------------------------------------------
+            // MMA issuer
+            // ------------------------------------------------------------------
+            constexpr uint32_t ID_S = idesc_bf16(128, BQ, false);          // S^T, dP^T
+            constexpr uint32_t ID_G = idesc_bf16(128, D, true);            // dV, dK
+            constexpr uint32_t ID_Q = idesc_bf16(128, BQ, true, true);     // dQ^T = K^T dS^T
+            const uint64_t k_kmaj = sdesc_sw128(sbase + X::OFF_K, 16, 1024);
+            const uint64_t v_kmaj = sdesc_sw128(sbase + X::OFF_V, 16, 1024);
+            const uint64_t k_mn = sdesc_sw128(sbase + X::OFF_K, X::KV_SLAB, 1024);
+            const uint64_t ds_kmaj = sdesc_sw128(sbase + X::OFF_DS, 16, 1024);
+            const uint64_t ds_mn = sdesc_sw128(sbase + X::OFF_DS, X::DS_SLAB, 1024);
+            bool ok = wait_phase(bar(X::B_KV_FULL), 0, wd, ROLE_MMA, blk_id);
+            tc_fence_after();
+
+            // dQ^T = K^T dS^T for step m: A = K MN-major (d x keys), B = dS^T
+            // MN-major (queries x keys), 16 keys per step, once the dQ warps
+            // have read dQ of step m-1.  With d on the TMEM lanes the dQ warps'
+            // reductions cover whole 128-byte lines.
+            auto dq_of = [&](int m) -> bool {
+                if (m >= 1 && !wait_phase(bar(X::B_DQ_EMPTY), (m - 1) & 1, wd, ROLE_MMA, blk_id))
+                    return false;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t off = uint32_t((kk * 2048) >> 4);
+                    mma_ss(tmem + X::TM_DQ, desc_add(k_mn, off), desc_add(ds_mn, off), ID_Q,
+                           kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(X::B_DQ_FULL));
+                return true;
+            };
+
+            for (int n = 0; ok && n < nsteps; ++n) {
+                const int s = n % NSX;
+                if (!wait_phase(bar(X::B_QD_FULL + s), (n / NSX) & 1, wd, ROLE_MMA, blk_id)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sq = sbase + X::OFF_Q + s * X::QD_BYTES;
+                const uint32_t sdo = sbase + X::OFF_DO + s * X::QD_BYTES;
+                const uint64_t q_kmaj = sdesc_sw128(sq, 16, 1024);
+                const uint64_t do_kmaj = sdesc_sw128(sdo, 16, 1024);
+                // S^T = K Q^T into X (dV(n-1), issued earlier, has read P(n-1)).
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t oa = uint32_t(((kk / 4) * X::KV_SLAB + (kk % 4) * 32) >> 4);
+                    const uint32_t ob = uint32_t(((kk / 4) * X::QD_SLAB + (kk % 4) * 32) >> 4);
+                    mma_ss(tmem + X::TM_X, desc_add(k_kmaj, oa), desc_add(q_kmaj, ob), ID_S,
+                           kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(X::B_S_FULL));
+                // The tensor core works on dQ of step n-1 while the compute
+                // warps take the exponentials of step n.
+                if (n >= 1 && !dq_of(n - 1)) {
+                    ok = false;
+                    break;
+                }
+                // dP^T = V dO^T into X once every compute warp has read S^T.
+                if (!wait_phase(bar(X::B_S_FREE), n & 1, wd, ROLE_MMA, blk_id)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t oa = uint32_t(((kk / 4) * X::KV_SLAB + (kk % 4) * 32) >> 4);
+                    const uint32_t ob = uint32_t(((kk / 4) * X::QD_SLAB + (kk % 4) * 32) >> 4);
+                    mma_ss(tmem + X::TM_X, desc_add(v_kmaj, oa), desc_add(do_kmaj, ob), ID_S,
+                           kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(X::B_DP_FULL));
+                // Once P (in X) and dS (shared memory) are written:
+                // dV += P^T dO: A = P from TMEM (queries 16kk.. at columns
+                // (kk/4)*64 + (kk%4)*8, see the compute warps), B = dO MN-major;
+                // dK += dS^T Q: A = dS K-major (keys x queries), B = Q MN-major
+                // (16 query rows of 128 bytes per step).
+                if (!wait_phase(bar(X::B_DS_READY), n & 1, wd, ROLE_MMA, blk_id)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t do_mn = sdesc_sw128(sdo, X::QD_SLAB, 1024);
+                const uint64_t q_mn = sdesc_sw128(sq, X::QD_SLAB, 1024);
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    mma_ts(tmem + X::TM_DV, tmem + X::TM_X + uint32_t((kk / 4) * 64 + (kk % 4) * 8),
+                           desc_add(do_mn, uint32_t((kk * 2048) >> 4)), ID_G,
+                           (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    mma_ss(tmem + X::TM_DK,
+                           desc_add(ds_kmaj, uint32_t(((kk / 4) * X::DS_SLAB + (kk % 4) * 32) >> 4)),
+                           desc_add(q_mn, uint32_t((kk * 2048) >> 4)), ID_G,
+                           (n > 0 || kk > 0) ? 1u : 0u);
+                // Q, dO (and -LSE2, -D, read before DS_READY) of step n are
+                // no longer needed: the producer may refill the stage.
+                tc_commit(bar(X::B_QD_EMPTY + s));
+            }
+            if (ok) ok = dq_of(nsteps - 1);
+            if (ok) tc_commit(bar(X::B_ACC_FULL));
+            // Drain: every MMA this thread issued has completed before TMEM is freed.
+            tc_commit(bar(X::B_DRAIN));
+            wait_drain(bar(X::B_DRAIN), 0, watchdog_ns);
+        }
+    } else if (warp >= DQ_WARP0) {
+        regs_dec<X::REGS_DQ>();
+        // ------------------------------------------------------------------
+        // dQ drain: TMEM (lane = d index, columns = the step's queries) ->
+        // fp32 reductions, a warp covering 32 consecutive d of one row.
+        // ------------------------------------------------------------------
+        const int qw = warp - DQ_WARP0;                       // lane quarter
+        const uint32_t lane_base = uint32_t(32 * qw) << 16;
+        const int t = 32 * qw + lane;
+        for (int n = 0; n < nsteps; ++n) {
+            if (!warp_wait(bar(X::B_DQ_FULL), n & 1, wd, ROLE_DQ, blk_id)) break;
+            tc_fence_after();
+            const int q0 = (qb_first + n) * BQ;
+            const int rows = min(BQ, N - q0);
+            float* base = dq_acc + ((long long)bh * Npad + q0) * D + t;
+#pragma unroll
+            for (int c = 0; c < BQ / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + X::TM_DQ + c * 32, r);
+                if (c == BQ / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(X::B_DQ_EMPTY));
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (c * 32 + j < rows)
+                        red_add_f32(base + (long long)(c * 32 + j) * D, __uint_as_float(r[j]));
+            }
+        }
+    } else {
+        regs_inc<X::REGS_COMPUTE>();
+        // ------------------------------------------------------------------
+        // Compute warps: key row r (TMEM lane), query columns half*64 ..
+        // half*64+63.
+        // ------------------------------------------------------------------
+        const int qw = warp % 4, half = warp / 4;
+        const int r = 32 * qw + lane;                         // key row in the block
+        const int key = k0 + r;
+        const uint32_t lane_base = uint32_t(32 * qw) << 16;
+        const uint32_t xcol = X::TM_X + uint32_t(half * 64);  // this warp's X columns
+        const float cs = scale * LOG2E;
+        bool ok = true;
+        for (int n = 0; ok && n < nsteps; ++n) {
+            const int s = n % NSX;
+            const int q0 = (qb_first + n) * BQ;
+            // QD_FULL: -LSE2 / -D of this block have landed; S_FULL: S^T in X.
+            if (!warp_wait(bar(X::B_QD_FULL + s), (n / NSX) & 1, wd, ROLE_COMPUTE, blk_id) ||
+                !warp_wait(bar(X::B_S_FULL), n & 1, wd, ROLE_COMPUTE, blk_id)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const bool need_mask = (causal && q0 < k0 + BK) || (q0 + BQ > N) || (k0 + BK > N);
+            const float* vl = reinterpret_cast<const float*>(smem + X::OFF_VEC + s * X::VEC_BYTES) +
+                              half * 64;
+            const float* vd = vl + BQ;
+            const int qi0 = q0 + half * 64;
+            float p[64];
+            {
+                uint32_t sv[64];
+                tmem_ld32(tmem + lane_base + xcol, *reinterpret_cast<uint32_t(*)[32]>(sv));
+                tmem_ld32(tmem + lane_base + xcol + 32,
+                          *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(X::B_S_FREE));
+                if (need_mask) {
+                    p_chunk<true>(sv, vl, cs, qi0, key, N, causal, p);
+                    p_chunk<true>(sv + 32, vl + 32, cs, qi0 + 32, key, N, causal, p + 32);
+                } else {
+                    p_chunk<false>(sv, vl, cs, qi0, key, N, causal, p);
+                    p_chunk<false>(sv + 32, vl + 32, cs, qi0 + 32, key, N, causal, p + 32);
+                }
+            }
+            // DP_FULL: dP^T in X; it also follows dK and dQ of step n-1, so
+            // the dS buffer is free.
+            if (!warp_wait(bar(X::B_DP_FULL), n & 1, wd, ROLE_COMPUTE, blk_id)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t sds = sbase + X::OFF_DS;
+            uint32_t dpv[64];
+            tmem_ld32(tmem + lane_base + xcol, *reinterpret_cast<uint32_t(*)[32]>(dpv));
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                if (c == 1)
+                    tmem_ld32(tmem + lane_base + xcol + 32,
+                              *reinterpret_cast<uint32_t(*)[32]>(dpv + 32));
+                uint32_t pu[16], du[16];
+                ds_chunk(p + c * 32, dpv + c * 32, vd + c * 32, pu, du);
+                // P over columns xcol + 16c .. +15: inside the dP^T columns
+                // this warp read first (xcol .. xcol+31), so no other warp's
+                // unread dP^T is overwritten.
+                tmem_st16(tmem + lane_base + xcol + uint32_t(c * 16), pu);
+                // dS row r, queries half*64 + 32c .. +31, 128-byte swizzled
+                // (16-byte chunk index XOR row % 8 inside 1 KiB atoms).
+                const uint32_t row_base = sds + half * X::DS_SLAB + (r / 8) * 1024 + (r % 8) * 128;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const uint32_t phys = uint32_t((c * 4 + k4) ^ (r % 8));
+                    st_shared_v4(row_base + phys * 16, du[4 * k4], du[4 * k4 + 1], du[4 * k4 + 2],
+                                 du[4 * k4 + 3]);
+                }
+            }
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(X::B_DS_READY));
+        }
+        // Epilogue: dV and scale * dK of this warp's rows and column half.
+        if (ok && warp_wait(bar(X::B_ACC_FULL), 0, wd, ROLE_COMPUTE, blk_id)) {
+            tc_fence_after();
+            constexpr int HC = D / 2;                         // columns per half
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t tcol = (which == 0 ? X::TM_DV : X::TM_DK) + half * HC;
+                const float mul = which == 0 ? 1.f : scale;
+                __nv_bfloat16* dst =
+                    (which == 0 ? dv + sdv.row(bh, H, key) : dk + sdk.row(bh, H, key)) + half * HC;
+#pragma unroll
+                for (int c = 0; c < HC / 32; ++c) {
+                    uint32_t x[32];
+                    tmem_ld32(tmem + lane_base + tcol + c * 32, x);
+                    if (key < N) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            uint4 w;
+                            w.x = pack_bf16x2(mul * __uint_as_float(x[8 * k4 + 0]),
+                                              mul * __uint_as_float(x[8 * k4 + 1]));
+                            w.y = pack_bf16x2(mul * __uint_as_float(x[8 * k4 + 2]),
+                                              mul * __uint_as_float(x[8 * k4 + 3]));
+                            w.z = pack_bf16x2(mul * __uint_as_float(x[8 * k4 + 4]),
+                                              mul * __uint_as_float(x[8 * k4 + 5]));
+                            w.w = pack_bf16x2(mul * __uint_as_float(x[8 * k4 + 6]),
+                                              mul * __uint_as_float(x[8 * k4 + 7]));
+                            d4[k4] = w;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    // Teardown: after every thread is done with TMEM, the allocating warp frees it.
+    tc_fence_before();
+    cta_sync_x();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, X::TM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 constexpr int kMaxDevices = 64;             // current_device() accepts indices below this
@@ -808,23 +1311,39 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
     auto enc = [&](CUtensorMap* m, const void* p, const St3& x, int rows) {
         return fa_internal::encode_bhnd_map(m, p, D, N, H, B, x.b, x.h, x.n, rows);
     };
-    if (enc(&mq, q, st[0], C::BQ) != FA_OK || enc(&mk, k, st[1], BK) != FA_OK ||
-        enc(&mv, v, st[2], BK) != FA_OK || enc(&mdo, dout, st[4], C::BQ) != FA_OK)
+    // d = 128 runs bwd_kernel_x (128 query rows per step), d = 64 bwd_kernel.
+    constexpr bool WIDE = D == 128;
+    constexpr int BQ = WIDE ? CfgX::BQ : C::BQ;
+    constexpr int ALLOC = WIDE ? CfgX::ALLOC : C::ALLOC;
+    if (enc(&mq, q, st[0], BQ) != FA_OK || enc(&mk, k, st[1], BK) != FA_OK ||
+        enc(&mv, v, st[2], BK) != FA_OK || enc(&mdo, dout, st[4], BQ) != FA_OK)
         return FA_ERR_UNSUPPORTED;
 
     // The dynamic shared-memory limit is a per-device function attribute: set
-    // once per (instantiation, device).
+    // once per (instantiation, device).  bwd_kernel_x's setmaxnreg split needs
+    // the launch to give every thread CfgX::REGS_LAUNCH registers: its
+    // compiled count is checked once per device as well.
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
+    static int regs[kMaxDevices];
     std::call_once(once[dev], [&] {
-        attr_err[dev] = cudaFuncSetAttribute(bwd_kernel<D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::ALLOC);
+        const void* fn;
+        if constexpr (WIDE)
+            fn = reinterpret_cast<const void*>(bwd_kernel_x);
+        else
+            fn = reinterpret_cast<const void*>(bwd_kernel<D>);
+        attr_err[dev] = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             ALLOC);
+        cudaFuncAttributes fa_attr{};
+        if (attr_err[dev] == cudaSuccess) attr_err[dev] = cudaFuncGetAttributes(&fa_attr, fn);
+        regs[dev] = fa_attr.numRegs;
     });
     cudaError_t e = attr_err[dev];
     if (e != cudaSuccess) {
         fa_internal::set_last_cuda_error(int(e));
         return FA_ERR_LAUNCH;
     }
+    if (WIDE && regs[dev] != CfgX::REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
 
     const long long prep_threads = BH * np * (D / 8);
     bwd_prep<D><<<unsigned((prep_threads + 255) / 256), 256, 0, stream>>>(
@@ -839,10 +1358,16 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
     const long long head_bytes = 12LL * np * D;
     long long hg = (48LL << 20) / head_bytes;
     hg = hg < 1 ? 1 : (hg > BH ? BH : hg);
-    bwd_kernel<D><<<unsigned(nkb * BH), NUM_THREADS, C::ALLOC, stream>>>(
-        mq, mk, mv, mdo, nlse2, ndvec, dq_acc, static_cast<__nv_bfloat16*>(dk),
-        static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, int(hg), wd_ns,
-        inject, st[6], st[7]);
+    if constexpr (WIDE)
+        bwd_kernel_x<<<unsigned(nkb * BH), CfgX::THREADS, CfgX::ALLOC, stream>>>(
+            mq, mk, mv, mdo, nlse2, ndvec, dq_acc, static_cast<__nv_bfloat16*>(dk),
+            static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, int(hg),
+            wd_ns, inject, st[6], st[7]);
+    else
+        bwd_kernel<D><<<unsigned(nkb * BH), NUM_THREADS, C::ALLOC, stream>>>(
+            mq, mk, mv, mdo, nlse2, ndvec, dq_acc, static_cast<__nv_bfloat16*>(dk),
+            static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, int(hg),
+            wd_ns, inject, st[6], st[7]);
     const long long out_threads = BH * N * (D / 8);
     bwd_dq_out<D><<<unsigned((out_threads + 255) / 256), 256, 0, stream>>>(
         dq_acc, static_cast<__nv_bfloat16*>(dq), BH, H, N, int(np), scale, st[5]);
