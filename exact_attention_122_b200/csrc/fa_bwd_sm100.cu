@@ -772,18 +772,19 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 // ---------------------------------------------------------------------------
 // d = 128 kernel: 128 query rows per step, every MMA at M = N = 128.
 //
-// TMEM holds dQ, dV and dK (128 columns each) and one 128-column region X
-// that serves, in turn, S^T of the step, dP^T of the step (once the compute
-// warps have read S^T), and P as bf16 pairs (written by each compute warp
-// over the dP^T columns it has already read).  K stays in shared memory, so
-// S^T = K Q^T and dP^T = V dO^T are SS products.  Per step n the MMA thread
-// issues
-//   S^T(n) | dQ(n-1) | (S^T read) dP^T(n) | (P, dS written) dV(n), dK(n)
-// so the compute warps' exponentials of step n overlap the tensor core's dQ
-// of step n-1 and dP^T of step n; dV(n), issued before S^T(n+1) that
-// overwrites X, has read P(n) first (MMAs from one thread run in issue
-// order); and the Q / dO stage of step n is released right after dK(n), a
-// whole step before the next S^T needs the refill.
+// TMEM holds dV and dK (128 columns each) and two 128-column regions:
+//   X  S^T of the step, then dP^T of the step once the compute warps have
+//      read S^T;
+//   Y  P of the step as bf16 pairs (64 columns, written by the compute
+//      warps once the dQ warps have read the previous dQ^T), then dQ^T of
+//      the step (the dQ MMA is issued after the dV MMA that reads P).
+// K stays in shared memory, so S^T = K Q^T and dP^T = V dO^T are SS
+// products.  Per step n the MMA thread issues
+//   (S^T(n) read) dP^T(n) | (dP^T(n) read) S^T(n+1) |
+//   (P, dS of step n written) dV(n), dK(n), dQ(n)
+// so the compute warps' exponentials of step n+1 run while the tensor core
+// works on the gradients of step n, and the Q / dO stage of step n is
+// released right after dK(n).
 // 512 threads: warps 0-7 compute, 8-11 dQ drain, 12 MMA, 13 TMA, 14-15 idle;
 // the compute warpgroups take 176 registers, the dQ warpgroup 64 and the
 // last warpgroup 88 (setmaxnreg, from 128 at launch).
@@ -825,15 +826,16 @@ struct CfgX {
     static constexpr int B_DQ_EMPTY = 6 + 2 * NSX;
     static constexpr int B_ACC_FULL = 7 + 2 * NSX;
     static constexpr int B_DRAIN = 8 + 2 * NSX;
-    static constexpr int NUM_BARS = 9 + 2 * NSX;
+    static constexpr int B_DP_FREE = 9 + 2 * NSX;
+    static constexpr int NUM_BARS = 10 + 2 * NSX;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem base, abort flag
     static constexpr int BYTES = OFF_MISC + 16;
     // The whole 227 KiB: what is left over after BYTES absorbs the rounding
     // of the dynamic shared-memory base up to 1 KiB (checked in the kernel).
     static constexpr int ALLOC = 227 * 1024;
     static_assert(BYTES <= ALLOC, "shared memory budget");
-    static constexpr uint32_t TM_X = 0;                  // S^T, then dP^T, then P
-    static constexpr uint32_t TM_DQ = 128;               // dQ^T: d on the lanes
+    static constexpr uint32_t TM_X = 0;                  // S^T, then dP^T
+    static constexpr uint32_t TM_DQ = 128;               // Y: P, then dQ^T (d on the lanes)
     static constexpr uint32_t TM_DV = 256;
     static constexpr uint32_t TM_DK = 384;
     static constexpr uint32_t TM_COLS = 512;
@@ -869,8 +871,7 @@ __device__ __forceinline__ void p_chunk(const uint32_t* sv, const float* nl, flo
 
 // ds = p * (dP - D) for 32 query columns; P and dS rounded to bf16 pairs.
 __device__ __forceinline__ void ds_chunk(const float* p, const uint32_t* dpv,
-                                         const float* nd, uint32_t (&pu)[16],
-                                         uint32_t (&du)[16]) {
+                                         const float* nd, uint32_t* pu, uint32_t (&du)[16]) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
         const float4 d4 = *reinterpret_cast<const float4*>(nd + j);
@@ -947,6 +948,7 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         mbar_init(bar(X::B_S_FULL), 1);
         mbar_init(bar(X::B_S_FREE), COMPUTE_WARPS);
         mbar_init(bar(X::B_DP_FULL), 1);
+        mbar_init(bar(X::B_DP_FREE), COMPUTE_WARPS);
         mbar_init(bar(X::B_DS_READY), COMPUTE_WARPS);
         mbar_init(bar(X::B_DQ_FULL), 1);
         mbar_init(bar(X::B_DQ_EMPTY), 4);
@@ -1026,36 +1028,13 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             bool ok = wait_phase(bar(X::B_KV_FULL), 0, wd, ROLE_MMA, blk_id);
             tc_fence_after();
 
-            // dQ^T = K^T dS^T for step m: A = K MN-major (d x keys), B = dS^T
-            // MN-major (queries x keys), 16 keys per step, once the dQ warps
-            // have read dQ of step m-1.  With d on the TMEM lanes the dQ warps'
-            // reductions cover whole 128-byte lines.
-            auto dq_of = [&](int m) -> bool {
-                if (m >= 1 && !wait_phase(bar(X::B_DQ_EMPTY), (m - 1) & 1, wd, ROLE_MMA, blk_id))
+            // S^T = K Q^T for step m into X: A = K K-major, B = Q K-major.
+            auto s_of = [&](int m) -> bool {
+                const int sm = m % NSX;
+                if (!wait_phase(bar(X::B_QD_FULL + sm), (m / NSX) & 1, wd, ROLE_MMA, blk_id))
                     return false;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk) {
-                    const uint32_t off = uint32_t((kk * 2048) >> 4);
-                    mma_ss(tmem + X::TM_DQ, desc_add(k_mn, off), desc_add(ds_mn, off), ID_Q,
-                           kk > 0 ? 1u : 0u);
-                }
-                tc_commit(bar(X::B_DQ_FULL));
-                return true;
-            };
-
-            for (int n = 0; ok && n < nsteps; ++n) {
-                const int s = n % NSX;
-                if (!wait_phase(bar(X::B_QD_FULL + s), (n / NSX) & 1, wd, ROLE_MMA, blk_id)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t sq = sbase + X::OFF_Q + s * X::QD_BYTES;
-                const uint32_t sdo = sbase + X::OFF_DO + s * X::QD_BYTES;
-                const uint64_t q_kmaj = sdesc_sw128(sq, 16, 1024);
-                const uint64_t do_kmaj = sdesc_sw128(sdo, 16, 1024);
-                // S^T = K Q^T into X (dV(n-1), issued earlier, has read P(n-1)).
+                const uint64_t q_kmaj = sdesc_sw128(sbase + X::OFF_Q + sm * X::QD_BYTES, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t oa = uint32_t(((kk / 4) * X::KV_SLAB + (kk % 4) * 32) >> 4);
@@ -1064,18 +1043,20 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                            kk > 0 ? 1u : 0u);
                 }
                 tc_commit(bar(X::B_S_FULL));
-                // The tensor core works on dQ of step n-1 while the compute
-                // warps take the exponentials of step n.
-                if (n >= 1 && !dq_of(n - 1)) {
-                    ok = false;
-                    break;
-                }
-                // dP^T = V dO^T into X once every compute warp has read S^T.
+                return true;
+            };
+            if (ok) ok = s_of(0);
+            for (int n = 0; ok && n < nsteps; ++n) {
+                const int s = n % NSX;
+                const uint32_t sq = sbase + X::OFF_Q + s * X::QD_BYTES;
+                const uint32_t sdo = sbase + X::OFF_DO + s * X::QD_BYTES;
+                // dP^T = V dO^T into X once every compute warp has read S^T(n).
                 if (!wait_phase(bar(X::B_S_FREE), n & 1, wd, ROLE_MMA, blk_id)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint64_t do_kmaj = sdesc_sw128(sdo, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t oa = uint32_t(((kk / 4) * X::KV_SLAB + (kk % 4) * 32) >> 4);
@@ -1084,11 +1065,20 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                            kk > 0 ? 1u : 0u);
                 }
                 tc_commit(bar(X::B_DP_FULL));
-                // Once P (in X) and dS (shared memory) are written:
-                // dV += P^T dO: A = P from TMEM (queries 16kk.. at columns
-                // (kk/4)*64 + (kk%4)*8, see the compute warps), B = dO MN-major;
-                // dK += dS^T Q: A = dS K-major (keys x queries), B = Q MN-major
-                // (16 query rows of 128 bytes per step).
+                // S^T(n+1) into X once every compute warp has read dP^T(n).
+                if (!wait_phase(bar(X::B_DP_FREE), n & 1, wd, ROLE_MMA, blk_id)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (n + 1 < nsteps && !s_of(n + 1)) {
+                    ok = false;
+                    break;
+                }
+                // Once P(n) (in Y) and dS(n) (shared memory) are written:
+                // dV += P^T dO: A = P from TMEM (16 queries = 8 columns per
+                // step), B = dO MN-major (16 query rows of 128 bytes);
+                // dK += dS^T Q: A = dS K-major (keys x queries), B = Q MN-major.
                 if (!wait_phase(bar(X::B_DS_READY), n & 1, wd, ROLE_MMA, blk_id)) {
                     ok = false;
                     break;
@@ -1098,7 +1088,7 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 const uint64_t q_mn = sdesc_sw128(sq, X::QD_SLAB, 1024);
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    mma_ts(tmem + X::TM_DV, tmem + X::TM_X + uint32_t((kk / 4) * 64 + (kk % 4) * 8),
+                    mma_ts(tmem + X::TM_DV, tmem + X::TM_DQ + uint32_t(kk * 8),
                            desc_add(do_mn, uint32_t((kk * 2048) >> 4)), ID_G,
                            (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
@@ -1110,8 +1100,19 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 // Q, dO (and -LSE2, -D, read before DS_READY) of step n are
                 // no longer needed: the producer may refill the stage.
                 tc_commit(bar(X::B_QD_EMPTY + s));
+                // dQ^T = K^T dS^T into Y (after the dV MMA that read P; the
+                // compute warps wrote P(n) only after the dQ warps had read
+                // dQ^T(n-1)): A = K MN-major (d x keys), B = dS^T MN-major
+                // (queries x keys), 16 keys per step.  With d on the TMEM
+                // lanes the dQ warps' reductions cover whole 128-byte lines.
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t off = uint32_t((kk * 2048) >> 4);
+                    mma_ss(tmem + X::TM_DQ, desc_add(k_mn, off), desc_add(ds_mn, off), ID_Q,
+                           kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(X::B_DQ_FULL));
             }
-            if (ok) ok = dq_of(nsteps - 1);
             if (ok) tc_commit(bar(X::B_ACC_FULL));
             // Drain: every MMA this thread issued has completed before TMEM is freed.
             tc_commit(bar(X::B_DRAIN));
@@ -1199,30 +1200,41 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 break;
             }
             tc_fence_after();
-            const uint32_t sds = sbase + X::OFF_DS;
-            uint32_t dpv[64];
-            tmem_ld32(tmem + lane_base + xcol, *reinterpret_cast<uint32_t(*)[32]>(dpv));
+            uint32_t pu[32];
+            {
+                uint32_t dpv[64];
+                tmem_ld32(tmem + lane_base + xcol, *reinterpret_cast<uint32_t(*)[32]>(dpv));
+                tmem_ld32(tmem + lane_base + xcol + 32,
+                          *reinterpret_cast<uint32_t(*)[32]>(dpv + 32));
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(X::B_DP_FREE));
+                const uint32_t sds = sbase + X::OFF_DS;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                if (c == 1)
-                    tmem_ld32(tmem + lane_base + xcol + 32,
-                              *reinterpret_cast<uint32_t(*)[32]>(dpv + 32));
-                uint32_t pu[16], du[16];
-                ds_chunk(p + c * 32, dpv + c * 32, vd + c * 32, pu, du);
-                // P over columns xcol + 16c .. +15: inside the dP^T columns
-                // this warp read first (xcol .. xcol+31), so no other warp's
-                // unread dP^T is overwritten.
-                tmem_st16(tmem + lane_base + xcol + uint32_t(c * 16), pu);
-                // dS row r, queries half*64 + 32c .. +31, 128-byte swizzled
-                // (16-byte chunk index XOR row % 8 inside 1 KiB atoms).
-                const uint32_t row_base = sds + half * X::DS_SLAB + (r / 8) * 1024 + (r % 8) * 128;
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t du[16];
+                    ds_chunk(p + c * 32, dpv + c * 32, vd + c * 32, pu + c * 16, du);
+                    // dS row r, queries half*64 + 32c .. +31, 128-byte swizzled
+                    // (16-byte chunk index XOR row % 8 inside 1 KiB atoms).
+                    const uint32_t row_base =
+                        sds + half * X::DS_SLAB + (r / 8) * 1024 + (r % 8) * 128;
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const uint32_t phys = uint32_t((c * 4 + k4) ^ (r % 8));
-                    st_shared_v4(row_base + phys * 16, du[4 * k4], du[4 * k4 + 1], du[4 * k4 + 2],
-                                 du[4 * k4 + 3]);
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const uint32_t phys = uint32_t((c * 4 + k4) ^ (r % 8));
+                        st_shared_v4(row_base + phys * 16, du[4 * k4], du[4 * k4 + 1],
+                                     du[4 * k4 + 2], du[4 * k4 + 3]);
+                    }
                 }
             }
+            // P(n) into Y (queries half*64 .. +63 at columns half*32 .. +31)
+            // once the dQ warps have read dQ^T(n-1) from there.
+            if (n >= 1 && !warp_wait(bar(X::B_DQ_EMPTY), (n - 1) & 1, wd, ROLE_COMPUTE, blk_id)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            tmem_st16(tmem + lane_base + X::TM_DQ + uint32_t(half * 32), pu);
+            tmem_st16(tmem + lane_base + X::TM_DQ + uint32_t(half * 32 + 16), pu + 16);
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
