@@ -775,9 +775,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 // TMEM holds dV and dK (128 columns each) and two 128-column regions:
 //   X  S^T of the step, then dP^T of the step once the compute warps have
 //      read S^T;
-//   Y  P of the step as bf16 pairs (64 columns, written by the compute
-//      warps once the dQ warps have read the previous dQ^T), then dQ^T of
-//      the step (the dQ MMA is issued after the dV MMA that reads P).
+//   Y  P of the step as bf16 pairs (columns 0-63, written by the compute
+//      warps once the dQ warps have read those columns of the previous
+//      dQ^T), then dQ^T of the step (the dQ MMA is issued after the dV MMA
+//      that reads P, and after the dQ warps have read all of the previous
+//      dQ^T).
 // K stays in shared memory, so S^T = K Q^T and dP^T = V dO^T are SS
 // products.  Per step n the MMA thread issues
 //   (S^T(n) read) dP^T(n) | (dP^T(n) read) S^T(n+1) |
@@ -786,8 +788,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 // works on the gradients of step n, and the Q / dO stage of step n is
 // released right after dK(n).
 // 512 threads: warps 0-7 compute, 8-11 dQ drain, 12 MMA, 13 TMA, 14-15 idle;
-// the compute warpgroups take 176 registers, the dQ warpgroup 64 and the
-// last warpgroup 88 (setmaxnreg, from 128 at launch).
+// the compute warpgroups take 176 registers, the dQ warpgroup 72 and the
+// last warpgroup 80 (setmaxnreg, from 128 at launch).
 // ---------------------------------------------------------------------------
 struct CfgX {
     static constexpr int D = 128;
@@ -796,8 +798,8 @@ struct CfgX {
     static constexpr int THREADS = 512;
     static constexpr int REGS_LAUNCH = 128;
     static constexpr int REGS_COMPUTE = 176;
-    static constexpr int REGS_DQ = 64;
-    static constexpr int REGS_OTHER = 88;
+    static constexpr int REGS_DQ = 72;
+    static constexpr int REGS_OTHER = 80;
     static_assert(256 * REGS_COMPUTE + 128 * REGS_DQ + 128 * REGS_OTHER <=
                       THREADS * REGS_LAUNCH,
                   "setmaxnreg split within the launch's registers");
@@ -827,7 +829,8 @@ struct CfgX {
     static constexpr int B_ACC_FULL = 7 + 2 * NSX;
     static constexpr int B_DRAIN = 8 + 2 * NSX;
     static constexpr int B_DP_FREE = 9 + 2 * NSX;
-    static constexpr int NUM_BARS = 10 + 2 * NSX;
+    static constexpr int B_DQ_LO_EMPTY = 10 + 2 * NSX;   // Y's P columns read
+    static constexpr int NUM_BARS = 11 + 2 * NSX;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem base, abort flag
     static constexpr int BYTES = OFF_MISC + 16;
     // The whole 227 KiB: what is left over after BYTES absorbs the rounding
@@ -952,6 +955,7 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         mbar_init(bar(X::B_DS_READY), COMPUTE_WARPS);
         mbar_init(bar(X::B_DQ_FULL), 1);
         mbar_init(bar(X::B_DQ_EMPTY), 4);
+        mbar_init(bar(X::B_DQ_LO_EMPTY), 4);
         mbar_init(bar(X::B_ACC_FULL), 1);
         mbar_init(bar(X::B_DRAIN), 1);
         *abort_flag = 0;
@@ -1100,11 +1104,16 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 // Q, dO (and -LSE2, -D, read before DS_READY) of step n are
                 // no longer needed: the producer may refill the stage.
                 tc_commit(bar(X::B_QD_EMPTY + s));
-                // dQ^T = K^T dS^T into Y (after the dV MMA that read P; the
-                // compute warps wrote P(n) only after the dQ warps had read
-                // dQ^T(n-1)): A = K MN-major (d x keys), B = dS^T MN-major
-                // (queries x keys), 16 keys per step.  With d on the TMEM
-                // lanes the dQ warps' reductions cover whole 128-byte lines.
+                // dQ^T = K^T dS^T into Y (after the dV MMA that read P, and
+                // once the dQ warps have read all of dQ^T(n-1)): A = K MN-major
+                // (d x keys), B = dS^T MN-major (queries x keys), 16 keys per
+                // step.  With d on the TMEM lanes the dQ warps' reductions
+                // cover whole 128-byte lines.
+                if (n >= 1 && !wait_phase(bar(X::B_DQ_EMPTY), (n - 1) & 1, wd, ROLE_MMA, blk_id)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
                     const uint32_t off = uint32_t((kk * 2048) >> 4);
@@ -1133,19 +1142,23 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             const int q0 = (qb_first + n) * BQ;
             const int rows = min(BQ, N - q0);
             float* base = dq_acc + ((long long)bh * Npad + q0) * D + t;
+            // Two halves of 64 queries: the first half's columns are where the
+            // compute warps put P of the next step, so they are released
+            // (DQ_LO_EMPTY) before any reduction is issued; the whole region
+            // (DQ_EMPTY) before the next dQ MMA.
 #pragma unroll
-            for (int c = 0; c < BQ / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_base + X::TM_DQ + c * 32, r);
-                if (c == BQ / 32 - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(X::B_DQ_EMPTY));
-                }
+            for (int hq = 0; hq < 2; ++hq) {
+                uint32_t r[64];
+                tmem_ld32(tmem + lane_base + X::TM_DQ + hq * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
+                tmem_ld32(tmem + lane_base + X::TM_DQ + hq * 64 + 32,
+                          *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(hq == 0 ? X::B_DQ_LO_EMPTY : X::B_DQ_EMPTY));
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (c * 32 + j < rows)
-                        red_add_f32(base + (long long)(c * 32 + j) * D, __uint_as_float(r[j]));
+                for (int j = 0; j < 64; ++j)
+                    if (hq * 64 + j < rows)
+                        red_add_f32(base + (long long)(hq * 64 + j) * D, __uint_as_float(r[j]));
             }
         }
     } else {
@@ -1228,7 +1241,7 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             }
             // P(n) into Y (queries half*64 .. +63 at columns half*32 .. +31)
             // once the dQ warps have read dQ^T(n-1) from there.
-            if (n >= 1 && !warp_wait(bar(X::B_DQ_EMPTY), (n - 1) & 1, wd, ROLE_COMPUTE, blk_id)) {
+            if (n >= 1 && !warp_wait(bar(X::B_DQ_LO_EMPTY), (n - 1) & 1, wd, ROLE_COMPUTE, blk_id)) {
                 ok = false;
                 break;
             }
