@@ -782,11 +782,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 //      dQ^T).
 // K stays in shared memory, so S^T = K Q^T and dP^T = V dO^T are SS
 // products.  Per step n the MMA thread issues
-//   (S^T(n) read) dP^T(n) | (dP^T(n) read) S^T(n+1) |
-//   (P, dS of step n written) dV(n), dK(n), dQ(n)
+//   (S^T(n) read) dP^T(n) | (P(n) in Y) dV(n) | (dP^T(n) read) S^T(n+1) |
+//   (dS(n) written) dK(n), dQ(n)
 // so the compute warps' exponentials of step n+1 run while the tensor core
-// works on the gradients of step n, and the Q / dO stage of step n is
-// released right after dK(n).
+// works on the gradients of step n, dV(n) runs while dS(n) is computed, and
+// the Q / dO stage of step n is released right after dK(n).
 // 512 threads: warps 0-7 compute, 8-11 dQ drain, 12 MMA, 13 TMA, 14-15 idle;
 // the compute warpgroups take 176 registers, the dQ warpgroup 72 and the
 // last warpgroup 80 (setmaxnreg, from 128 at launch).
@@ -830,7 +830,8 @@ struct CfgX {
     static constexpr int B_DRAIN = 8 + 2 * NSX;
     static constexpr int B_DP_FREE = 9 + 2 * NSX;
     static constexpr int B_DQ_LO_EMPTY = 10 + 2 * NSX;   // Y's P columns read
-    static constexpr int NUM_BARS = 11 + 2 * NSX;
+    static constexpr int B_P_READY = 11 + 2 * NSX;       // P of the step in Y
+    static constexpr int NUM_BARS = 12 + 2 * NSX;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem base, abort flag
     static constexpr int BYTES = OFF_MISC + 16;
     // The whole 227 KiB: what is left over after BYTES absorbs the rounding
@@ -872,9 +873,9 @@ __device__ __forceinline__ void p_chunk(const uint32_t* sv, const float* nl, flo
     }
 }
 
-// ds = p * (dP - D) for 32 query columns; P and dS rounded to bf16 pairs.
+// ds = p * (dP - D) for 32 query columns, rounded to bf16 pairs.
 __device__ __forceinline__ void ds_chunk(const float* p, const uint32_t* dpv,
-                                         const float* nd, uint32_t* pu, uint32_t (&du)[16]) {
+                                         const float* nd, uint32_t (&du)[16]) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
         const float4 d4 = *reinterpret_cast<const float4*>(nd + j);
@@ -886,8 +887,6 @@ __device__ __forceinline__ void ds_chunk(const float* p, const uint32_t* dpv,
         float ds[4];
         f2_unpack(f2_mul(f2_pack(p[j], p[j + 1]), t01), ds[0], ds[1]);
         f2_unpack(f2_mul(f2_pack(p[j + 2], p[j + 3]), t23), ds[2], ds[3]);
-        pu[j / 2] = pack_bf16x2(p[j], p[j + 1]);
-        pu[j / 2 + 1] = pack_bf16x2(p[j + 2], p[j + 3]);
         du[j / 2] = pack_bf16x2(ds[0], ds[1]);
         du[j / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
     }
@@ -956,6 +955,7 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         mbar_init(bar(X::B_DQ_FULL), 1);
         mbar_init(bar(X::B_DQ_EMPTY), 4);
         mbar_init(bar(X::B_DQ_LO_EMPTY), 4);
+        mbar_init(bar(X::B_P_READY), COMPUTE_WARPS);
         mbar_init(bar(X::B_ACC_FULL), 1);
         mbar_init(bar(X::B_DRAIN), 1);
         *abort_flag = 0;
@@ -1069,6 +1069,20 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                            kk > 0 ? 1u : 0u);
                 }
                 tc_commit(bar(X::B_DP_FULL));
+                // dV += P^T dO once P(n) is in Y: A = P from TMEM (16 queries =
+                // 8 columns per step), B = dO MN-major (16 query rows of 128
+                // bytes).
+                if (!wait_phase(bar(X::B_P_READY), n & 1, wd, ROLE_MMA, blk_id)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t do_mn = sdesc_sw128(sdo, X::QD_SLAB, 1024);
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    mma_ts(tmem + X::TM_DV, tmem + X::TM_DQ + uint32_t(kk * 8),
+                           desc_add(do_mn, uint32_t((kk * 2048) >> 4)), ID_G,
+                           (n > 0 || kk > 0) ? 1u : 0u);
                 // S^T(n+1) into X once every compute warp has read dP^T(n).
                 if (!wait_phase(bar(X::B_DP_FREE), n & 1, wd, ROLE_MMA, blk_id)) {
                     ok = false;
@@ -1079,22 +1093,14 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                     ok = false;
                     break;
                 }
-                // Once P(n) (in Y) and dS(n) (shared memory) are written:
-                // dV += P^T dO: A = P from TMEM (16 queries = 8 columns per
-                // step), B = dO MN-major (16 query rows of 128 bytes);
-                // dK += dS^T Q: A = dS K-major (keys x queries), B = Q MN-major.
+                // Once dS(n) is in shared memory: dK += dS^T Q: A = dS K-major
+                // (keys x queries), B = Q MN-major.
                 if (!wait_phase(bar(X::B_DS_READY), n & 1, wd, ROLE_MMA, blk_id)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t do_mn = sdesc_sw128(sdo, X::QD_SLAB, 1024);
                 const uint64_t q_mn = sdesc_sw128(sq, X::QD_SLAB, 1024);
-#pragma unroll
-                for (int kk = 0; kk < BQ / 16; ++kk)
-                    mma_ts(tmem + X::TM_DV, tmem + X::TM_DQ + uint32_t(kk * 8),
-                           desc_add(do_mn, uint32_t((kk * 2048) >> 4)), ID_G,
-                           (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
                     mma_ss(tmem + X::TM_DK,
@@ -1206,6 +1212,26 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                     p_chunk<false>(sv + 32, vl + 32, cs, qi0 + 32, key, N, causal, p + 32);
                 }
             }
+            // P(n) into Y (queries half*64 .. +63 at columns half*32 .. +31)
+            // once the dQ warps have read those columns of dQ^T(n-1); the dV
+            // MMA can then start before dP^T(n) is read.
+            {
+                uint32_t pu[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) pu[i] = pack_bf16x2(p[2 * i], p[2 * i + 1]);
+                if (n >= 1 &&
+                    !warp_wait(bar(X::B_DQ_LO_EMPTY), (n - 1) & 1, wd, ROLE_COMPUTE, blk_id)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                tmem_st16(tmem + lane_base + X::TM_DQ + uint32_t(half * 32), pu);
+                tmem_st16(tmem + lane_base + X::TM_DQ + uint32_t(half * 32 + 16), pu + 16);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(X::B_P_READY));
+            }
             // DP_FULL: dP^T in X; it also follows dK and dQ of step n-1, so
             // the dS buffer is free.
             if (!warp_wait(bar(X::B_DP_FULL), n & 1, wd, ROLE_COMPUTE, blk_id)) {
@@ -1213,7 +1239,6 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 break;
             }
             tc_fence_after();
-            uint32_t pu[32];
             {
                 uint32_t dpv[64];
                 tmem_ld32(tmem + lane_base + xcol, *reinterpret_cast<uint32_t(*)[32]>(dpv));
@@ -1226,7 +1251,7 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     uint32_t du[16];
-                    ds_chunk(p + c * 32, dpv + c * 32, vd + c * 32, pu + c * 16, du);
+                    ds_chunk(p + c * 32, dpv + c * 32, vd + c * 32, du);
                     // dS row r, queries half*64 + 32c .. +31, 128-byte swizzled
                     // (16-byte chunk index XOR row % 8 inside 1 KiB atoms).
                     const uint32_t row_base =
@@ -1239,15 +1264,6 @@ bwd_kernel_x(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                     }
                 }
             }
-            // P(n) into Y (queries half*64 .. +63 at columns half*32 .. +31)
-            // once the dQ warps have read dQ^T(n-1) from there.
-            if (n >= 1 && !warp_wait(bar(X::B_DQ_LO_EMPTY), (n - 1) & 1, wd, ROLE_COMPUTE, blk_id)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            tmem_st16(tmem + lane_base + X::TM_DQ + uint32_t(half * 32), pu);
-            tmem_st16(tmem + lane_base + X::TM_DQ + uint32_t(half * 32 + 16), pu + 16);
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
