@@ -15,7 +15,9 @@
 //   bwd_prep     D_i and LSE_i * log2(e) per row into the workspace (padded
 //                rows get D = 0, LSE = +inf, so their P is 0), and zeroes
 //                the fp32 dQ accumulator.
-//   bwd_kernel   one CTA per 128-key block of one (batch, head), 448 threads:
+//   bwd_kernel_x (d = 128, below) or
+//   bwd_kernel   (d = 64) one CTA per 128-key block of one (batch, head),
+//                448 threads:
 //                  warps 0-7   compute: P, dS for the key block's 128 rows
 //                              (warp w: TMEM lane quarter w % 4, half of the
 //                              query columns w / 4)
@@ -34,6 +36,8 @@
 //                block i-1's gradients are issued after block i's S^T and
 //                dP^T, so the compute warps' exponentials for block i overlap
 //                the tensor core's work on block i-1.
+//                bwd_kernel_x keeps the same division of work with 128
+//                query rows per step and its own TMEM plan (see there).
 //   bwd_dq_out   dQ = bf16(scale * accumulator).
 //
 // Every mbarrier wait is bounded by a %globaltimer watchdog, as in the
@@ -73,9 +77,11 @@ constexpr float LOG2E = 1.4426950408889634f;
 enum : uint32_t { ROLE_COMPUTE = 1u, ROLE_MMA = 2u, ROLE_PRODUCER = 3u, ROLE_DQ = 4u,
                   ROLE_DRAIN = 5u };
 
-// D = 128: 64 query rows per step and dQ^T (d on the TMEM lanes, M = 128).
-// D = 64:  128 query rows per step and dQ (queries on the lanes, M = 128).
-// Both keep every MMA at M = 128 and fit the 512 TMEM columns.
+// bwd_kernel's layout.  D = 64 (the head dimension it runs): 128 query rows
+// per step and dQ (queries on the lanes, M = 128).  D = 128 (64 query rows
+// per step, dQ^T with d on the TMEM lanes) is kept for the template but no
+// longer launched: d = 128 runs bwd_kernel_x.  Both keep every MMA at M = 128
+// and fit the 512 TMEM columns.
 template <int D>
 struct Cfg {
     static constexpr int BQ = D == 128 ? 64 : 128;
