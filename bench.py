@@ -681,8 +681,8 @@ def run_bwd(args):
             "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s",
                          "frac": value / peak,
                          "traffic": load_traffic(w.name + "_bwd", BWD_KERNEL_SOURCE),
-                         "traffic_kernel": "bwd_kernel", "peak_source": peak_src,
-                         "kernel": "bwd_prep + bwd_kernel + bwd_dq_out (whole step)"},
+                         "traffic_kernel": "bwd_kernel_x", "peak_source": peak_src,
+                         "kernel": "bwd_prep + bwd_kernel_x + bwd_dq_out (whole step)"},
             "gpu_launches": 3 * args.steps, "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
     return 0
