@@ -1443,7 +1443,10 @@ fa_status fa_get_device_status(void* stream, unsigned* detail) {
                                                                            : FA_ERR_LAUNCH;
     }
     if (detail) *detail = word;
-    return word == 0 ? FA_OK : FA_ERR_TIMEOUT;
+    if (word == 0) return FA_OK;
+    // The top byte holds the status the kernel recorded.
+    const unsigned code = word >> 24;
+    return code == unsigned(FA_ERR_LAUNCH) ? FA_ERR_LAUNCH : FA_ERR_TIMEOUT;
 }
 
 const char* fa_status_string(int status) {

@@ -399,9 +399,12 @@ fa_status fa_fwd_debug(const void* q, const void* k, const void* v, void* o, flo
 
 /*
  * fa_get_device_status -- read and clear the device status word of the
- * current device.  Synchronises `stream` first.  Returns FA_OK or
- * FA_ERR_TIMEOUT (a kernel watchdog fired since the last read); *detail, if
- * not NULL, receives the raw word (role and unit of the first timeout).
+ * current device.  Synchronises `stream` first.  Returns FA_OK, or the
+ * status a kernel recorded since the last read: FA_ERR_TIMEOUT (a watchdog
+ * fired), or FA_ERR_LAUNCH (the d = 128 backward kernel found its dynamic
+ * shared memory placed so that its 226 KiB layout did not fit, and returned
+ * without writing dK or dV).  *detail, if not NULL, receives the raw word:
+ * status << 24 | role << 20 | unit (or CTA) of the first event.
  * Returns FA_ERR_NO_DEVICE / FA_ERR_LAUNCH if the CUDA calls fail.
  *
  * The word is one per device (one for the forward kernels, one for the
