@@ -77,15 +77,13 @@ constexpr float LOG2E = 1.4426950408889634f;
 enum : uint32_t { ROLE_COMPUTE = 1u, ROLE_MMA = 2u, ROLE_PRODUCER = 3u, ROLE_DQ = 4u,
                   ROLE_DRAIN = 5u };
 
-// bwd_kernel's layout.  D = 64 (the head dimension it runs): 128 query rows
-// per step and dQ (queries on the lanes, M = 128).  D = 128 (64 query rows
-// per step, dQ^T with d on the TMEM lanes) is kept for the template but no
-// longer launched: d = 128 runs bwd_kernel_x.  Both keep every MMA at M = 128
-// and fit the 512 TMEM columns.
+// bwd_kernel's layout (d = 64; d = 128 runs bwd_kernel_x): 128 query rows per
+// step and dQ with the queries on the TMEM lanes; every MMA at M = 128, within
+// the 512 TMEM columns.
 template <int D>
 struct Cfg {
-    static constexpr int BQ = D == 128 ? 64 : 128;
-    static constexpr bool DQ_T = D == 128;
+    static_assert(D == 64, "bwd_kernel runs d = 64 only");
+    static constexpr int BQ = 128;
     static constexpr int KV_BYTES = BK * D * 2;
     static constexpr int KV_SLAB = BK * 128;             // 64 columns of a K/V tile
     static constexpr int QD_BYTES = BQ * D * 2;
@@ -125,7 +123,7 @@ struct Cfg {
     static constexpr uint32_t TM_DP = BQ;
     static constexpr uint32_t TM_DQ = 2 * BQ;                  // dQ^T: BQ cols; dQ: D cols
     static constexpr uint32_t TM_P = TM_DQ;
-    static constexpr uint32_t DQ_COLS = DQ_T ? BQ : D;
+    static constexpr uint32_t DQ_COLS = D;
     static constexpr uint32_t TM_K = TM_DQ + DQ_COLS;
     static constexpr uint32_t TM_DV = TM_K + D / 2;
     static constexpr uint32_t TM_DK = TM_DV + D;
@@ -470,8 +468,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_bf16(128, BQ, false);          // S^T, dP^T
             constexpr uint32_t ID_G = idesc_bf16(128, D, true);            // dV, dK
-            constexpr uint32_t ID_Q = C::DQ_T ? idesc_bf16(128, BQ, true, true)   // dQ^T
-                                              : idesc_bf16(128, D, true, true);   // dQ
+            constexpr uint32_t ID_Q = idesc_bf16(128, D, true, true);      // dQ = dS K
             const uint64_t dV_kmaj = sdesc_sw128(sbase + C::OFF_V, 16, 1024);
             const uint64_t dK_mn = sdesc_sw128(sbase + C::OFF_K, C::KV_SLAB, 1024);
             bool ok = wait_phase(bar(C::B_KV_FULL), 0, wd, ROLE_MMA, blk_id) &&
@@ -511,12 +508,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
                     const uint32_t off = uint32_t((kk * 2048) >> 4);
-                    if (C::DQ_T)   // dQ^T = K^T dS^T: A = K MN-major (d x keys), B = dS^T MN-major
-                        mma_ss(tmem + C::TM_DQ, desc_add(dK_mn, off), desc_add(ds_mn, off), ID_Q,
-                               kk > 0 ? 1u : 0u);
-                    else           // dQ = dS K: A = dS MN-major (queries x keys), B = K MN-major
-                        mma_ss(tmem + C::TM_DQ, desc_add(ds_mn, off), desc_add(dK_mn, off), ID_Q,
-                               kk > 0 ? 1u : 0u);
+                    // dQ = dS K: A = dS MN-major (queries x keys), B = K MN-major
+                    mma_ss(tmem + C::TM_DQ, desc_add(ds_mn, off), desc_add(dK_mn, off), ID_Q,
+                           kk > 0 ? 1u : 0u);
                 }
                 // One commit for the block's gradients: the dQ warps, which
                 // wait on it every step, pass the release of the dS buffer and
@@ -584,25 +578,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 mbar_arrive(bar(C::B_QD_EMPTY + (n % NS)));
             }
             const int q0 = (qb_first + n) * BQ;
-            if (C::DQ_T) {
-                // lane = d index t; columns = the BQ queries of the block
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tmem + lane_base + C::TM_DQ, r0);
-                tmem_ld32(tmem + lane_base + C::TM_DQ + 32, r1);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
-                const int t = 32 * qw + lane;
-                float* base = dq_acc + ((long long)bh * Npad + q0) * D + t;
-                const int rows = min(BQ, N - q0);
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (j < rows) red_add_f32(base + (long long)j * D, __uint_as_float(r0[j]));
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (32 + j < rows)
-                        red_add_f32(base + (long long)(32 + j) * D, __uint_as_float(r1[j]));
-            } else {
+            {
                 // lane = query row; columns = d
                 uint32_t r0[32], r1[32];
                 tmem_ld32(tmem + lane_base + C::TM_DQ, r0);
@@ -1345,7 +1321,7 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N,
                  const St3 (&st)[8], int causal, float scale, unsigned char* ws,
                  cudaStream_t stream, int dev, unsigned long long wd_ns, int inject) {
-    using C = Cfg<D>;
+    using C = Cfg<64>;                 // bwd_kernel's layout (the d = 64 path)
     const long long BH = (long long)B * H;
     const long long np = npad_of(N);
     const WsLayout wl = ws_layout(BH, N, D);
@@ -1378,7 +1354,7 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
         if constexpr (WIDE)
             fn = reinterpret_cast<const void*>(bwd_kernel_x);
         else
-            fn = reinterpret_cast<const void*>(bwd_kernel<D>);
+            fn = reinterpret_cast<const void*>(bwd_kernel<64>);
         attr_err[dev] = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              ALLOC);
         cudaFuncAttributes fa_attr{};
@@ -1411,7 +1387,7 @@ fa_status launch(const void* q, const void* k, const void* v, const void* o, con
             static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, int(hg),
             wd_ns, inject, st[6], st[7]);
     else
-        bwd_kernel<D><<<unsigned(nkb * BH), NUM_THREADS, C::ALLOC, stream>>>(
+        bwd_kernel<64><<<unsigned(nkb * BH), NUM_THREADS, C::ALLOC, stream>>>(
             mq, mk, mv, mdo, nlse2, ndvec, dq_acc, static_cast<__nv_bfloat16*>(dk),
             static_cast<__nv_bfloat16*>(dv), int(BH), H, N, int(np), causal, scale, int(hg),
             wd_ns, inject, st[6], st[7]);
