@@ -97,7 +97,12 @@ struct Cfg {
     static constexpr int OFF_DO = OFF_Q + NS * QD_BYTES;
     static constexpr int OFF_DS = OFF_DO + NS * QD_BYTES;
     static constexpr int OFF_VEC = OFF_DS + 2 * DS_BYTES;
-    static constexpr int OFF_BAR = OFF_VEC + NS * VEC_BYTES;
+    // dQ staging: per dQ warp 16 rows of d fp32, rows 16 bytes apart beyond
+    // their length so the row-per-lane stores hit distinct banks.
+    static constexpr int STG_ROW = D * 4 + 16;
+    static constexpr int STG_WARP = 16 * STG_ROW;
+    static constexpr int OFF_STG = OFF_VEC + NS * VEC_BYTES;
+    static constexpr int OFF_BAR = OFF_STG + 4 * STG_WARP;
     static constexpr int B_KV_FULL = 0;
     static constexpr int B_QD_FULL = 1;                  // [NS]
     static constexpr int B_QD_EMPTY = 1 + NS;            // [NS]
@@ -579,25 +584,45 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             }
             const int q0 = (qb_first + n) * BQ;
             {
-                // lane = query row; columns = d
+                // lane = query row; columns = d.  The rows go through shared
+                // memory, 16 at a time, so the reductions are issued with lane
+                // = column: each instruction covers 128 contiguous bytes of one
+                // row (a lane per row would touch 32 rows in 16-byte pieces).
                 uint32_t r0[32], r1[32];
                 tmem_ld32(tmem + lane_base + C::TM_DQ, r0);
                 tmem_ld32(tmem + lane_base + C::TM_DQ + 32, r1);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(C::B_DQ_EMPTY));
-                const int row = q0 + 32 * qw + lane;
-                if (row < N) {
-                    float* base = dq_acc + ((long long)bh * Npad + row) * D;
+                const uint32_t stg = sbase + C::OFF_STG + qw * C::STG_WARP;
+                const int rows = min(32, N - (q0 + 32 * qw));      // valid rows of this warp
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        red_add_v4_f32(base + j, __uint_as_float(r0[j]), __uint_as_float(r0[j + 1]),
-                                       __uint_as_float(r0[j + 2]), __uint_as_float(r0[j + 3]));
+                for (int hr = 0; hr < 2; ++hr) {
+                    if ((lane >> 4) == hr) {
+                        const uint32_t dst = stg + (lane & 15) * C::STG_ROW;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        red_add_v4_f32(base + 32 + j, __uint_as_float(r1[j]),
-                                       __uint_as_float(r1[j + 1]), __uint_as_float(r1[j + 2]),
-                                       __uint_as_float(r1[j + 3]));
+                        for (int j = 0; j < 32; j += 4) {
+                            st_shared_v4(dst + j * 4, r0[j], r0[j + 1], r0[j + 2], r0[j + 3]);
+                            st_shared_v4(dst + 128 + j * 4, r1[j], r1[j + 1], r1[j + 2], r1[j + 3]);
+                        }
+                    }
+                    __syncwarp();
+#pragma unroll 4
+                    for (int i = 0; i < 16; ++i) {
+                        const int lr = 16 * hr + i;               // row within the warp's 32
+                        if (lr < rows) {
+                            float a, c;
+                            asm volatile("ld.shared.f32 %0, [%1];"
+                                         : "=f"(a) : "r"(stg + i * C::STG_ROW + lane * 4));
+                            asm volatile("ld.shared.f32 %0, [%1];"
+                                         : "=f"(c) : "r"(stg + i * C::STG_ROW + 128 + lane * 4));
+                            float* base =
+                                dq_acc + ((long long)bh * Npad + q0 + 32 * qw + lr) * D + lane;
+                            red_add_f32(base, a);
+                            red_add_f32(base + 32, c);
+                        }
+                    }
+                    __syncwarp();
                 }
             }
         }
