@@ -172,6 +172,41 @@ def test_peaked_scores_rescale_often(fa, d):
         check(o, lse, O_ref, L_ref, f"peaked d={d} causal={causal}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_extreme_scores_one_hot(fa, d):
+    """Q, K ~ N(0, 20^2): scaled scores with a spread of hundreds, so every
+    softmax row is one-hot to within bf16 and the running maximum jumps by far
+    more than the lazy-rescale threshold from tile to tile."""
+    q, k, v = synth.draw_qkv(1, 2, 1000, d, seed=77, qk_std=20.0)
+    scale = 1.0 / math.sqrt(d)
+    for causal in (True, False):
+        o, lse = run(fa, q, k, v, causal, scale)
+        O_ref, L_ref = oracle.attention_fp64(q, k, v, causal=causal, scale=scale)
+        check(o, lse, O_ref, L_ref, f"one-hot d={d} causal={causal}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_equal_scores_give_prefix_means(fa, d):
+    """Q = 0: every score is 0, so P is uniform over the allowed keys and row
+    i of O is the mean of v_0..v_i (causal) or of all v (not causal), and
+    LSE_i = ln(#allowed keys) -- closed forms, checked directly as well as
+    against the oracle."""
+    N = 777
+    _, k, v = synth.draw_qkv(1, 2, N, d, seed=78)
+    q = torch.zeros_like(k)
+    for causal in (True, False):
+        o, lse = run(fa, q, k, v, causal, 1.0 / math.sqrt(d))
+        V = f64(v)
+        if causal:
+            counts = np.arange(1, N + 1, dtype=np.float64)
+            O_ref = np.cumsum(V, axis=2) / counts[None, None, :, None]
+            L_ref = np.broadcast_to(np.log(counts), (1, 2, N))
+        else:
+            O_ref = np.broadcast_to(V.mean(axis=2, keepdims=True), V.shape)
+            L_ref = np.full((1, 2, N), math.log(N))
+        check(o, lse, O_ref, L_ref, f"equal scores d={d} causal={causal}")
+
+
 def test_many_short_units(fa):
     """More units than SMs, each short: exercises the persistent unit loop."""
     q, k, v = synth.draw_qkv(2, 150, 256, 64, seed=5)
