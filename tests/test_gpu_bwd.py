@@ -112,6 +112,31 @@ def test_bwd_nonstandard_scale(fa):
     compare_all(fa, 2, 2, 300, 64, False, seed=45, scale=0.37)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_bwd_equal_scores_closed_forms(fa, d):
+    """Q = 0: every score is 0 and P is uniform over the allowed keys, so
+    dK = scale dS^T Q is exactly zero, and dV_j is the sum of dO_i / (number
+    of keys row i sees) over the rows i that see key j -- closed forms,
+    independent of the oracle.  dQ is compared with the oracle."""
+    B, H, N = 1, 2, 640
+    _, k, v = synth.draw_qkv(B, H, N, d, seed=91)
+    q = torch.zeros_like(k)
+    do = synth.draw_dout(B, H, N, d, seed=91)
+    scale = 1 / math.sqrt(d)
+    DO = do.double().numpy()
+    for causal in (True, False):
+        dq, dk, dv = gpu_grads(fa, q, k, v, do, causal, scale)
+        assert float(dk.abs().max()) == 0.0, f"dK of Q = 0 must vanish (causal={causal})"
+        if causal:
+            w = DO / np.arange(1, N + 1, dtype=np.float64)[None, None, :, None]
+            dv_ref = np.flip(np.cumsum(np.flip(w, axis=2), axis=2), axis=2)
+        else:
+            dv_ref = np.broadcast_to(DO.sum(axis=2, keepdims=True) / N, DO.shape)
+        check_grad(dv, dv_ref, f"dV equal scores d={d} causal={causal}")
+        dq_ref, _, _, _ = oracle.attention_bwd_fp64(q, k, v, do, causal=causal, scale=scale)
+        check_grad(dq, dq_ref, f"dQ equal scores d={d} causal={causal}")
+
+
 def test_bwd_causal_row0_and_sums(fa):
     """Properties of the exact gradients: causal query 0 has dQ = 0 (its only
     key has weight 1); the keys' dV sum to the queries' dO sum (every P row
