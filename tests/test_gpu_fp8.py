@@ -187,6 +187,31 @@ def test_fp8_full_size_sampled(fa):
     assert float(np.sqrt(np.mean(e * e))) <= REL_RMS * float(np.sqrt(np.mean(r * r)))
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_equal_scores_give_prefix_means(fa, d):
+    """Q = 0 (E4M3 zero bytes): every score is 0 and every P is exactly 1 in
+    E4M3, so O is the prefix mean (causal) or the mean of the decoded V, up to
+    fp32 accumulation and the bf16 output (2^-8 relative), and LSE = ln(#keys)."""
+    N = 900
+    (_, k8, v8), sc = synth.draw_qkv_fp8(1, 2, N, d, seed=96)
+    q8 = torch.zeros_like(k8)
+    V = deq(v8, sc[2])
+    vmax = float(np.abs(V).max())
+    for causal in (True, False):
+        o, lse = run(fa, q8, k8, v8, sc, causal, 1 / math.sqrt(d))
+        O = o.float().cpu().numpy().astype(np.float64)
+        L = lse.cpu().numpy().astype(np.float64)
+        if causal:
+            counts = np.arange(1, N + 1, dtype=np.float64)
+            O_ref = np.cumsum(V, axis=2) / counts[None, None, :, None]
+        else:
+            counts = np.full(N, float(N))
+            O_ref = np.broadcast_to(V.mean(axis=2, keepdims=True), V.shape)
+        bound = 2.0 ** -8 * np.abs(O_ref) + 1e-5 * vmax
+        assert float((np.abs(O - O_ref) / bound).max()) <= 1.0, f"d={d} causal={causal}"
+        assert float(np.abs(L - np.log(counts)[None, None, :]).max()) <= TOL_LSE
+
+
 def test_fp8_deterministic(fa):
     (q8, k8, v8), sc = synth.draw_qkv_fp8(1, 4, 1536, 128, seed=65)
     a = run(fa, q8, k8, v8, sc, True, 0.0883883)

@@ -430,6 +430,27 @@ def test_decode_matches_square_last_rows(fa, Nq):
     assert float((l_dec - l_sq[:, :, N - Nq:]).abs().max()) <= TOL_LSE
 
 
+@pytest.mark.parametrize("Nq,causal", [(1, False), (7, True), (16, True), (100, True)])
+def test_decode_equal_scores_give_means(fa, Nq, causal):
+    """Q = 0 against N_k keys: each row's O is the mean of the V rows it may
+    see (causal: keys j <= i + N_k - N_q) and LSE = ln(that count), closed
+    forms checked directly."""
+    Nk, d = 3001, 128
+    _, k, v = synth.draw_qkv(1, 2, Nk, d, seed=95)
+    q = torch.zeros(1, 2, Nq, d, dtype=torch.bfloat16)
+    qd, kd, vd = (t.to("cuda:0") for t in (q, k, v))
+    o, lse = fa.fa_fwd_decode(qd, kd, vd, causal=causal)
+    torch.cuda.synchronize()
+    st, word = fa.device_status()
+    assert st == fa.FA_OK, f"device status {fa.status_string(st)} {word:#x}"
+    V = f64(v)
+    csum = np.cumsum(V, axis=2)
+    counts = np.array([(i + Nk - Nq + 1) if causal else Nk for i in range(Nq)], dtype=np.float64)
+    O_ref = np.stack([csum[:, :, int(c) - 1] / c for c in counts], axis=2)
+    L_ref = np.broadcast_to(np.log(counts), (1, 2, Nq))
+    check(o, lse, O_ref, L_ref, f"decode equal scores Nq={Nq} causal={causal}")
+
+
 def test_decode_full_size_sampled(fa):
     """decode_32k (B=16, H=32, one query against 32768 keys, d=128) in the
     launch configuration `bench.py --decode` times: automatic split count and
