@@ -118,15 +118,24 @@ struct Layout {
     static constexpr int B_DRAIN = B_O_EMPTY + 2;
     static constexpr int B_UFULL = B_DRAIN + 1;      // [2] unit queue (dynamic schedule)
     static constexpr int B_UEMPTY = B_UFULL + 2;     // [2]
-    static constexpr int NUM_BARS = B_UEMPTY + 2;
+    static constexpr int B_S_FREE = B_UEMPTY + 2;    // [2] S_t read into registers (SEP_P)
+    static constexpr int B_PV_DONE = B_S_FREE + 2;   // [2] P_t V complete (SEP_P)
+    static constexpr int NUM_BARS = B_PV_DONE + 2;
     // tmem base, abort flag, zero flag, spare, unit queue slots [2]
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int OFF_UNIT = OFF_MISC + 16;
     static constexpr int BYTES = OFF_MISC + 32;
     static constexpr int ALLOC = BYTES + 1024;       // slack to align the base to 1 KiB
-    // TMEM columns
-    static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+    // TMEM columns.  SEP_P (bf16, d = 64): P_t gets its own 64 columns
+    // instead of overwriting S_t, so S_t of the next K/V tile can be computed
+    // while the softmax of the current one runs (S 2 x 128 + P 2 x 64 + O
+    // 2 x 64 = 512 columns).  Otherwise P_t aliases the first columns of S_t.
+    static constexpr bool SEP_P = D == 64 && !F8;
+    static constexpr uint32_t TM_S0 = 0, TM_S1 = 128;
+    static constexpr uint32_t TM_P0 = SEP_P ? 256 : TM_S0, TM_P1 = SEP_P ? 320 : TM_S1;
+    static constexpr uint32_t TM_O0 = SEP_P ? 384 : 256, TM_O1 = TM_O0 + D;
     static constexpr uint32_t TM_COLS = 512;
+    static_assert(TM_O1 + D <= TM_COLS, "TMEM columns");
     static_assert(ALLOC <= 227 * 1024, "shared memory budget");
     static_assert(BYTES > 116 * 1024, "one CTA per SM keeps TMEM allocation uncontended");
 };
@@ -346,11 +355,11 @@ __device__ __forceinline__ void exp_row_to_p(const float (&s)[BN], float scale_l
 // of the reference m and of O in TMEM, P into TMEM over S, publication of P on
 // p_bar, then the row sums.  a: the sub-tile's first row; row: this thread's
 // row.
-template <int D, bool F8>
-__device__ __forceinline__ void softmax_tile(float (&s)[BN], int j, int nkb, int Nk, int causal,
+template <int D, bool F8, typename PreP>
+__device__ __forceinline__ bool softmax_tile(float (&s)[BN], int j, int nkb, int Nk, int causal,
                                              int a, int row, int koff, float scale_log2, float& m,
-                                             float& l, float& lc, uint32_t tS, uint32_t tO,
-                                             uint32_t p_bar) {
+                                             float& l, float& lc, uint32_t tP, uint32_t tO,
+                                             uint32_t p_bar, PreP&& pre_p) {
     // Mask: keys beyond N_k on the last tile; causal: keys past
     // the row's limit on the tiles that cross the sub-tile's
     // first limit (the diagonal).
@@ -382,12 +391,15 @@ __device__ __forceinline__ void softmax_tile(float (&s)[BN], int j, int nkb, int
                                     fmax3(mx8[3], mx8[4], mx8[5]), mx8[6]),
                               mx8[7]);
     const float m_blk = s_top * scale_log2;
+    // With P in its own columns, the previous tile's P V may still be running:
+    // pre_p waits for it before O is rescaled or P overwritten.
+    if (!pre_p()) return false;
     // Lazy rescale: the reference m (that l and O refer to) moves
     // to the row's new maximum only when some row of the warp
     // exceeds it by more than rescale_log2 (first tile: m = -inf,
     // so every lane moves).  O is then rescaled in TMEM: the P V
-    // of tile j-1 is complete, its commit preceded the S_t commit
-    // waited on above.
+    // of tile j-1 is complete (P over S: its commit preceded the
+    // S_t commit waited on by the caller; P apart: pre_p waited).
     if (__any_sync(0xffffffffu, m_blk > m + rescale_log2<F8>())) {
         const float m_new = fmaxf(m, m_blk);
         const float alpha = ex2(m - m_new);      // 0 on the first tile
@@ -409,7 +421,7 @@ __device__ __forceinline__ void softmax_tile(float (&s)[BN], int j, int nkb, int
         m = m_new;
     }
     uint64_t acc[4] = {0, 0, 0, 0};              // four packed (0.f, 0.f)
-    exp_row_to_p<F8>(s, scale_log2, -m, acc, tS);
+    exp_row_to_p<F8>(s, scale_log2, -m, acc, tP);
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(p_bar);
@@ -432,6 +444,7 @@ __device__ __forceinline__ void softmax_tile(float (&s)[BN], int j, int nkb, int
         f2_unpack(acc[3], a6, a7);
         l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
     }
+    return true;
 }
 
 // Epilogue of one row: O / (l + lc) -> bf16 -> the row of o_head (element
@@ -549,6 +562,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(bar(L::B_P_FULL + t), BM);
             mbar_init(bar(L::B_O_FULL + t), 1);
             mbar_init(bar(L::B_O_EMPTY + t), BM);
+            mbar_init(bar(L::B_S_FREE + t), BM);
+            mbar_init(bar(L::B_PV_DONE + t), 1);
         }
         mbar_init(bar(L::B_DRAIN), 1);
         for (int i = 0; i < 2; ++i) {
@@ -694,6 +709,91 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 issue_pv<F8>(tO, tS, v_desc, ID_PV, first);
                 return true;
             };
+            if constexpr (L::SEP_P) {
+            // P apart from S: per K/V tile j, S_0(j+1) and S_1(j+1) go out as
+            // soon as each softmax warpgroup has read S_t(j) (S_FREE), ahead
+            // of O_0 += P_0 V_j and O_1 += P_1 V_j; each P V is committed to
+            // PV_DONE_t, which the softmax waits for before it writes the
+            // next P_t or rescales O_t.  K_{j+1} is used before V_j: both
+            // stages are found from the fill count (K_j, V_j, K_{j+1}, ...).
+            const uint32_t tP0 = tmem + L::TM_P0, tP1 = tmem + L::TM_P1;
+            uint32_t sc0 = 0, sc1 = 0;              // S_t issued over the CTA's lifetime
+            auto issue_s = [&](int t, uint32_t& sc, uint32_t sK, int u) -> bool {
+                if (sc > 0 &&
+                    !wait_phase(bar(L::B_S_FREE + t), (sc - 1) & 1u, wd, ROLE_MMA, u))
+                    return false;
+                tc_fence_after();
+                issue_qk<L::QK_STEPS, L::HALF_BYTES, F8>(t ? tS1 : tS0, t ? dq1 : dq0,
+                                                         desc_add(dk0, sK * stage_step), ID_S);
+                tc_commit(bar(L::B_S_FULL + t));
+                ++sc;
+                return true;
+            };
+            for (int kq = 0; ok; ++kq, ++units) {
+                const int u = next_unit_consumer(kq, ok, ROLE_MMA);
+                if (u < 0) break;
+                const Unit w = decode_unit(u, Nq, Nk, causal);
+                if (!wait_phase(bar(L::B_Q_FULL), units & 1u, wd, ROLE_MMA, u)) { ok = false; break; }
+                const uint32_t sK0 = cons % NS;
+                if (!wait_phase(bar(L::B_KV_FULL + sK0), (cons / NS) & 1u, wd, ROLE_MMA, u)) {
+                    ok = false;
+                    break;
+                }
+                ++cons;
+                if (!issue_s(0, sc0, sK0, u) || !issue_s(1, sc1, sK0, u)) { ok = false; break; }
+                tc_commit(bar(L::B_KV_EMPTY + sK0));
+                issued = true;
+                if (w.nb1 == 1) tc_commit(bar(L::B_Q_EMPTY));
+                for (int j = 0; j < w.nb1; ++j) {
+                    const bool next = j + 1 < w.nb1;
+                    const uint32_t cV = cons, cK = cons + 1;
+                    cons += next ? 2u : 1u;
+                    if (next) {
+                        const uint32_t sK = cK % NS;
+                        if (!wait_phase(bar(L::B_KV_FULL + sK), (cK / NS) & 1u, wd, ROLE_MMA, u)) {
+                            ok = false;
+                            break;
+                        }
+                        if (j + 1 < w.nb0 && !issue_s(0, sc0, sK, u)) { ok = false; break; }
+                        if (!issue_s(1, sc1, sK, u)) { ok = false; break; }
+                        tc_commit(bar(L::B_KV_EMPTY + sK));
+                        if (j + 1 == w.nb1 - 1) tc_commit(bar(L::B_Q_EMPTY));
+                    }
+                    const uint32_t sV = cV % NS;
+                    if (!wait_phase(bar(L::B_KV_FULL + sV), (cV / NS) & 1u, wd, ROLE_MMA, u)) {
+                        ok = false;
+                        break;
+                    }
+                    if (j < w.nb0) {
+                        if (j == 0 && !wait_phase(bar(L::B_O_EMPTY + 0), (units & 1u) ^ 1u, wd,
+                                                  ROLE_MMA, u)) {
+                            ok = false;
+                            break;
+                        }
+                        if (!pv(0, pcnt0, tO0, tP0, desc_add(dv0, sV * stage_step), j == 0, u)) {
+                            ok = false;
+                            break;
+                        }
+                        ++pcnt0;
+                        tc_commit(bar(L::B_PV_DONE + 0));
+                        if (j == w.nb0 - 1) tc_commit(bar(L::B_O_FULL + 0));
+                    }
+                    if (j == 0 && !wait_phase(bar(L::B_O_EMPTY + 1), (units & 1u) ^ 1u, wd,
+                                              ROLE_MMA, u)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!pv(1, pcnt1, tO1, tP1, desc_add(dv0, sV * stage_step), j == 0, u)) {
+                        ok = false;
+                        break;
+                    }
+                    ++pcnt1;
+                    tc_commit(bar(L::B_PV_DONE + 1));
+                    tc_commit(bar(L::B_KV_EMPTY + sV));
+                    if (j == w.nb1 - 1) tc_commit(bar(L::B_O_FULL + 1));
+                }
+            }
+            } else {
             for (int kq = 0; ok; ++kq, ++units) {
                 const int u = next_unit_consumer(kq, ok, ROLE_MMA);
                 if (u < 0) break;
@@ -779,6 +879,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (j == w.nb1 - 1) tc_commit(bar(L::B_O_FULL + 1));
                 }
             }
+            }
             if (issued) {
                 // Every MMA this thread issued must finish before TMEM is
                 // freed; on the normal path the softmax warps have already
@@ -807,6 +908,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int wr = (warp & 3) * 32 + lane;       // row within the sub-tile
         const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + (t == 0 ? L::TM_S0 : L::TM_S1);
+        const uint32_t tP = tmem + lane_base + (t == 0 ? L::TM_P0 : L::TM_P1);
         const uint32_t tO = tmem + lane_base + (t == 0 ? L::TM_O0 : L::TM_O1);
         uint32_t scnt = 0, ocnt = 0;
         bool ok = true;
@@ -821,6 +923,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             float l = 0.f;                           // running sum of exponentials
             float lc = 0.f;                          // rounding correction of l for O
             for (int j = 0; j < nb; ++j) {
+                const uint32_t k = scnt;             // this sub-tile's tile count so far
                 bool got = wait_phase(bar(L::B_S_FULL + t), scnt & 1u, wd, ROLE_SOFTMAX, u);
                 ++scnt;
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -832,8 +935,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(r[c]);
                 }
-                softmax_tile<D, F8>(s, j, nkb, Nk, causal, a, row, koff, scale_log2, m, l, lc, tS,
-                                    tO, bar(L::B_P_FULL + t));
+                if constexpr (L::SEP_P) {
+                    // S_t is in registers: the MMA thread may overwrite it
+                    tc_fence_before();
+                    mbar_arrive(bar(L::B_S_FREE + t));
+                }
+                auto pre_p = [&]() -> bool {
+                    if constexpr (L::SEP_P) {
+                        if (k == 0) return true;
+                        const bool done = wait_phase(bar(L::B_PV_DONE + t), (k - 1) & 1u, wd,
+                                                     ROLE_SOFTMAX, u);
+                        if (!__all_sync(0xffffffffu, done)) return false;
+                        tc_fence_after();
+                    }
+                    return true;
+                };
+                if (!softmax_tile<D, F8>(s, j, nkb, Nk, causal, a, row, koff, scale_log2, m, l, lc,
+                                         tP, tO, bar(L::B_P_FULL + t), pre_p)) {
+                    ok = false;
+                    break;
+                }
             }
             if (!ok) break;
             // Epilogue: O / l -> bf16 -> global; LSE.
