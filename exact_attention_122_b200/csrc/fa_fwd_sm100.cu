@@ -24,7 +24,7 @@
 //              through an NS-stage shared-memory ring
 //   warps 10-11 idle (they complete the third warpgroup)
 // The third warpgroup gives registers to the softmax warpgroups with
-// setmaxnreg (REGS_SOFTMAX / REGS_OTHER below).
+// setmaxnreg (Regs<D, F8>::SOFTMAX / OTHER below).
 // Each softmax thread owns one query row (TMEM lane == row), so the row max
 // and row sum are in-thread.  S_t (fp32, 128 columns) and O_t (fp32, d
 // columns) live in TMEM; P_t is written back as bf16 over the first 64
@@ -67,14 +67,19 @@ constexpr int MMA_WARP = 8;
 constexpr int TMA_WARP = 9;
 // Register split.  The launch gives every thread REGS_LAUNCH registers
 // (65536 / 384, rounded down to 8 and to the sub-partition share: 168).
-// Warpgroup 2 drops to REGS_OTHER once at the start and never rises again;
-// warpgroups 0 and 1 rise to REGS_SOFTMAX.  The sum must not exceed the
+// Warpgroup 2 drops to Regs::OTHER once at the start and never rises again;
+// warpgroups 0 and 1 rise to Regs::SOFTMAX.  The sum must not exceed the
 // launch total or setmaxnreg.inc never returns.
 constexpr int REGS_LAUNCH = 168;
-constexpr int REGS_SOFTMAX = 208;
-constexpr int REGS_OTHER = 80;
-static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER <= NUM_THREADS * REGS_LAUNCH,
-              "register split exceeds the launch allocation");
+// The bf16 d = 128 kernel spilled registers (ptxas -v) with 80 for the third
+// warpgroup; with 96 there and 200 for the softmax warpgroups it does not.
+template <int D, bool F8>
+struct Regs {
+    static constexpr int SOFTMAX = (D == 128 && !F8) ? 200 : 208;
+    static constexpr int OTHER = (D == 128 && !F8) ? 96 : 80;
+    static_assert(2 * 128 * SOFTMAX + 128 * OTHER <= NUM_THREADS * REGS_LAUNCH,
+                  "register split exceeds the launch allocation");
+};
 constexpr int SW_COLS = 64;        // bf16 elements per 128-byte swizzled row
 // Lazy rescale: the running max that l and O refer to is only moved when a
 // row's new maximum exceeds it by more than rescale_log2<F8> (log2 units), so
@@ -588,7 +593,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // Each role's code sits inside the branch that set its register budget,
     // so ptxas allocates it against that budget.
     if (warp >= 8) {
-    regs_dec<REGS_OTHER>();
+    regs_dec<Regs<D, F8>::OTHER>();
     if (warp >= 10) {
         // idle warps of the third warpgroup
     } else if (warp == TMA_WARP) {
@@ -903,7 +908,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // ------------------------------------------------------------------
         // Softmax warpgroups.  Thread = query row; TMEM lane = row.
         // ------------------------------------------------------------------
-        regs_inc<REGS_SOFTMAX>();
+        regs_inc<Regs<D, F8>::SOFTMAX>();
         const int t = warp >> 2;                     // sub-tile 0 or 1
         const int wr = (warp & 3) * 32 + lane;       // row within the sub-tile
         const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
