@@ -28,9 +28,11 @@
 // Each softmax thread owns one query row (TMEM lane == row), so the row max
 // and row sum are in-thread.  S_t (fp32, 128 columns) and O_t (fp32, d
 // columns) live in TMEM; P_t is written back as bf16 over the first 64
-// columns of S_t and read from TMEM by the PV MMA.  The two warpgroups
-// alternate with the single MMA issuer, so the tensor core works on one
-// sub-tile while the other sub-tile's exponentials run.
+// columns of S_t (bf16 d = 64: into 64 columns of its own) and read from
+// TMEM by the PV MMA.  The two warpgroups alternate with the single MMA
+// issuer, so the tensor core works on one sub-tile while the other
+// sub-tile's exponentials run; with P in its own columns the next tile's
+// S_t is issued as soon as the softmax has read the current one.
 //
 // Every mbarrier wait is bounded by a %globaltimer watchdog.  A wait that
 // runs out records FA_ERR_TIMEOUT in g_fa_status, raises a CTA-wide abort
